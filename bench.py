@@ -1,0 +1,445 @@
+"""Benchmark of the PR-Sink per-block step on B200.
+
+One step = one block of a 480x480 stream through 40 attention layers (heads 40 x 128): the
+fingerprint and pose retrieval with the dynamic-sink fill of every layer, then per layer the 3
+denoising passes and the Clean KV Update pass (KV append into ring slot b mod 3 + PR-Sink
+attention over ref 900 + static 2700 + dynamic 2700 + 3 x 2700 ring = 14400 keys), then the bank
+update.  The bank (M = 5) is filled during the first 20 blocks, which run untimed before the
+warm-up; the timed blocks are the steady state after it is frozen.
+
+Metric: blocks/s per 40-head layer (layer-blocks per second over all GPUs), with the attention
+TFLOP/s and its fraction of the measured dense bf16 peak.  Inputs are synthetic (N(0,1) bf16
+Q/K/V, clustered synthetic poses); per-layer caches are 295 MB and 40 layers are cycled, so
+every launch reads from HBM (the working set is far above the 126 MB L2).
+
+``--impl reference`` times the float64 CPU oracle on a bounded sample of the same workload.
+Under torchrun every rank runs its own stream (weak scaling, no data-path collective).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "PR-Sink attention TFLOPS (% of bf16 peak) and blocks/s per 40-head layer at 1 B200"
+UNIT = "layer-blocks/s"
+PASSES = 4          # 3 denoising passes + the Clean KV Update pass
+M_BANK = 5
+WRITE_BLOCKS = 20
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return dict(hbm=float(d["hbm_gbs"]), bf16=float(d["bf16_tflops"]),
+                    bf16_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                    source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = max(smax, float(parts[2]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return None
+        loaded = [v for v in sm if v > 0.5 * smax] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------------------------
+# our arm
+# ------------------------------------------------------------------------------------------
+
+def run_ours(args, rank: int, world: int, local_rank: int):
+    import torch
+    import torch.distributed as dist
+
+    import pose_retrieved_kv_b200 as P
+    import synth
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    cfg = synth.preset(args.config)
+    n_layers = args.layers
+    H, d = cfg["n_heads"], cfg["head_dim"]
+    st = P.PRSinkStream(cfg, n_layers=n_layers, M=M_BANK, write_blocks=WRITE_BLOCKS, device=dev)
+    lblk, T = st.L_blk, st.T
+    # a pool of distinct per-pass inputs (well above L2), reused round-robin over layer-passes
+    pool = args.pool
+    qkv = [[synth.normal_bf16((lblk, H, d), 100 + rank * 1000 + i, j).to(dev) for j in range(3)]
+           for i in range(pool)]
+    for layer in range(n_layers):
+        kr = synth.normal_bf16((st.L_ref, H, d), 7 + layer, 1).to(dev)
+        st.set_ref(layer, kr, kr)
+    n_blocks = WRITE_BLOCKS + args.warmup + args.steps
+    kp_all, ok_all, _ = synth.pose_stream(11 + rank, n_blocks)
+    kp_dev = torch.from_numpy(np.ascontiguousarray(kp_all[:, :, :62, :])).to(dev)
+    ok_dev = torch.from_numpy(ok_all).to(dev)
+    out = torch.empty((lblk, H, d), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    attn_events = []
+
+    def block(b, timed):
+        st.begin_block(kp_dev[b], ok_dev[b])
+        i = 0
+        for layer in range(n_layers):
+            for p in range(PASSES):
+                q, kn, vn = qkv[(b * n_layers * PASSES + i) % pool]
+                i += 1
+                lay = st.layout()
+                k, v = st.kv(layer)
+                P.prsink_kv_append(lay, kn, vn, k, v, P.SLOT_RING0 + st.b % st.R)
+                if p == PASSES - 1 and st.b == 0:
+                    P.prsink_kv_append(lay, kn, vn, k, v, P.SLOT_STATIC)
+                if timed:
+                    e0 = torch.cuda.Event(enable_timing=True)
+                    e1 = torch.cuda.Event(enable_timing=True)
+                    e0.record(stream)
+                P.prsink_attention(lay, q, k, v, out, None, st.dyn_src)
+                if timed:
+                    e1.record(stream)
+                    attn_events.append((e0, e1))
+        st.end_block()
+
+    for b in range(WRITE_BLOCKS + args.warmup):          # bank fill + warm-up, untimed
+        block(b, False)
+    torch.cuda.synchronize()
+    if P.prsink_sync_status() != P.PRSINK_OK:
+        raise RuntimeError("device status reported a timeout during warm-up")
+
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    n0 = P.prsink_launch_count()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for k in range(args.steps):
+        block(WRITE_BLOCKS + args.warmup + k, True)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    launches = P.prsink_launch_count() - n0
+    clk = clocks.stop()
+    ms = t0.elapsed_time(t1)
+    if P.prsink_sync_status() != P.PRSINK_OK:
+        raise RuntimeError("device status reported a timeout in the timed region")
+    attn_ms = [a.elapsed_time(b) for a, b in attn_events]
+    if world > 1:
+        tt = torch.tensor([ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, st, qkv, kp_all, ok_all, dev, world)
+
+    if rank != 0:
+        return None
+    peaks = _peaks()
+    layer_blocks = n_layers * args.steps * world
+    value = layer_blocks / (ms / 1e3)
+    flops = 4.0 * lblk * T * d * H                      # QK^T + PV, steady state: all keys valid
+    attn_avg_ms = statistics.mean(attn_ms)
+    achieved = flops / (attn_avg_ms / 1e3) / 1e12
+    peak = peaks["bf16_sustained"]
+    res = {
+        "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (N(0,1) bf16 Q/K/V, clustered synthetic poses; no weights needed)",
+        "config": {"workload": f"per-block step {args.config}: {n_layers} layers x "
+                               f"({PASSES - 1} denoise + 1 clean) x (append + PR-Sink attention), "
+                               "retrieval + dynamic fill, bank update",
+                   "heads": H, "head_dim": d, "queries": lblk, "keys": T,
+                   "ring_slots": cfg["ring_slots"], "layers": n_layers, "bank": M_BANK,
+                   "l2": "inputs larger than L2 (295 MB cache per layer, layers cycled)",
+                   "parallelism": f"replica x{world} (independent streams)"},
+        "attention": {"avg_ms": round(attn_avg_ms, 4), "tflops": round(achieved, 1),
+                      "frac_of_bf16_peak": round(achieved / peak, 4),
+                      "launches_timed": len(attn_ms)},
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
+                     "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": None,
+                     "peak_source": f"{peaks['source']} bf16_tflops_sustained"},
+        "gpu_launches": int(launches),
+        "clocks": clk,
+    }
+    if e2e is not None:
+        res["e2e"] = e2e
+    if not args.no_cpu_baseline and world == 1:
+        res["cpu_baseline"] = cpu_baseline(args, cfg)
+    return res
+
+
+def run_e2e(args, st, qkv, kp_all, ok_all, dev, world):
+    """Same step through the public API with pinned HOST inputs and outputs: every step copies
+    its poses and per-pass Q/K/V from the host and reads every attention output back.  Copies
+    run on their own streams, overlapped with compute through double buffering."""
+    import torch
+    import torch.distributed as dist
+
+    import pose_retrieved_kv_b200 as P
+
+    n_layers, pool = st.n_layers, len(qkv)
+    lblk = st.L_blk
+    H, d = st.cfg["n_heads"], st.cfg["head_dim"]
+    host_in = [[t.cpu().pin_memory() for t in s] for s in qkv]
+    host_out = [torch.empty((lblk, H, d), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    kp_h = torch.from_numpy(np.ascontiguousarray(kp_all[:, :, :62, :])).pin_memory()
+    ok_h = torch.from_numpy(ok_all).pin_memory()
+    stage = [[torch.empty((lblk, H, d), dtype=torch.bfloat16, device=dev) for _ in range(3)]
+             for _ in range(2)]
+    outs = [torch.empty((lblk, H, d), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    kp_d = torch.empty((3, 62, 3), dtype=torch.float32, device=dev)
+    ok_d = torch.empty(3, dtype=torch.uint8, device=dev)
+    comp = torch.cuda.current_stream(dev)
+    h2d = torch.cuda.Stream(dev)
+    d2h = torch.cuda.Stream(dev)
+    in_ready = [torch.cuda.Event() for _ in range(2)]
+    in_free = [torch.cuda.Event() for _ in range(2)]
+    out_ready = [torch.cuda.Event() for _ in range(2)]
+    out_free = [torch.cuda.Event() for _ in range(2)]
+    for e in in_free + out_free:
+        e.record(comp)
+    bytes_in = bytes_out = 0
+    first = WRITE_BLOCKS + args.warmup + args.steps
+    n_blocks = kp_all.shape[0]
+
+    def block(b):
+        nonlocal bytes_in, bytes_out
+        bb = b % n_blocks
+        with torch.cuda.stream(h2d):
+            kp_d.copy_(kp_h[bb], non_blocking=True)
+            ok_d.copy_(ok_h[bb], non_blocking=True)
+        comp.wait_stream(h2d)
+        bytes_in += kp_d.numel() * 4 + 3
+        st.begin_block(kp_d, ok_d)
+        i = 0
+        for layer in range(n_layers):
+            for p in range(PASSES):
+                j = i & 1
+                src = host_in[(b * n_layers * PASSES + i) % pool]
+                h2d.wait_event(in_free[j])
+                with torch.cuda.stream(h2d):
+                    for t, h in zip(stage[j], src):
+                        t.copy_(h, non_blocking=True)
+                    in_ready[j].record(h2d)
+                bytes_in += 3 * lblk * H * d * 2
+                comp.wait_event(in_ready[j])
+                comp.wait_event(out_free[j])
+                q, kn, vn = stage[j]
+                st.layer_pass(layer, q, kn, vn, outs[j], clean=(p == PASSES - 1))
+                in_free[j].record(comp)
+                out_ready[j].record(comp)
+                d2h.wait_event(out_ready[j])
+                with torch.cuda.stream(d2h):
+                    host_out[j].copy_(outs[j], non_blocking=True)
+                    out_free[j].record(d2h)
+                bytes_out += lblk * H * d * 2
+                i += 1
+        st.end_block()
+
+    for k in range(2):
+        block(first + k)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    bytes_in = bytes_out = 0
+    t0 = time.perf_counter()
+    for k in range(args.steps):
+        block(first + 2 + k)
+    torch.cuda.synchronize()
+    el = time.perf_counter() - t0
+    if world > 1:
+        tt = torch.tensor([el], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        el = float(tt.item())
+    if P.prsink_sync_status() != P.PRSINK_OK:
+        raise RuntimeError("device status reported a timeout in the e2e run")
+    return {"value": round(n_layers * args.steps * world / el, 3), "unit": UNIT,
+            "h2d_bytes_per_step": bytes_in // args.steps,
+            "d2h_bytes_per_step": bytes_out // args.steps}
+
+
+# ------------------------------------------------------------------------------------------
+# CPU oracle (baseline only)
+# ------------------------------------------------------------------------------------------
+
+def _cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def oracle_sample_seconds_per_layer_block(cfg, heads: int, seed: int = 0):
+    """Time the oracle on ``heads`` heads of one attention pass plus one append, and scale to
+    one layer-block (all heads, 4 passes)."""
+    import oracle
+    import synth
+
+    s = oracle.layout_sizes(cfg)
+    H, d = cfg["n_heads"], cfg["head_dim"]
+    sub = dict(cfg, n_heads=heads, block_index=1000, valid_mask=0xFF)
+    q = synth.normal_bf16((s["L_blk"], heads, d), seed, 0).double().numpy()
+    k = synth.normal_bf16((heads, s["T"], d), seed, 1).double().numpy()
+    v = synth.normal_bf16((heads, s["T"], d), seed, 2).double().numpy()
+    kn = synth.normal_bf16((s["L_blk"], heads, d), seed, 3).double().numpy()
+    t0 = time.perf_counter()
+    k2, v2 = oracle.kv_append(sub, kn, kn, k, v, oracle.SLOT_RING0)
+    oracle.attention(sub, q, k2, v2)
+    el = time.perf_counter() - t0
+    return el * (H / heads) * PASSES, el
+
+
+def cpu_baseline(args, cfg):
+    heads = args.cpu_heads
+    per_lb, el = oracle_sample_seconds_per_layer_block(cfg, heads)
+    return {"value": round(1.0 / per_lb, 6), "unit": UNIT, "cores": _cores(), "kind": "oracle",
+            "sample": f"{heads} of {cfg['n_heads']} heads, 1 pass (append + attention, all "
+                      f"{oracle_rows(cfg)} queries x {oracle_keys(cfg)} keys) in {el:.1f} s, "
+                      f"scaled x{cfg['n_heads'] // heads} heads x{PASSES} passes"}
+
+
+def oracle_rows(cfg):
+    return cfg["frames_per_block"] * cfg["grid_h"] * cfg["grid_w"]
+
+
+def oracle_keys(cfg):
+    lf = cfg["grid_h"] * cfg["grid_w"]
+    return lf * cfg["ref_frames"] + (2 + cfg["ring_slots"]) * cfg["frames_per_block"] * lf
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    import synth
+    cfg = synth.preset(args.config)
+    heads = args.cpu_heads
+    for _ in range(args.warmup):
+        oracle_sample_seconds_per_layer_block(cfg, 1)
+    per = []
+    t0 = time.perf_counter()
+    for k in range(args.steps):
+        per.append(oracle_sample_seconds_per_layer_block(cfg, heads, seed=k)[0])
+    wall = time.perf_counter() - t0
+    value = 1.0 / statistics.mean(per)
+    cb = {"value": round(value, 6), "unit": UNIT, "cores": _cores(), "kind": "oracle",
+          "sample": f"each step: {heads} of {cfg['n_heads']} heads, 1 pass, scaled to one "
+                    f"layer-block (x{cfg['n_heads'] // heads} heads x{PASSES} passes)"}
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(1e3 * wall / args.steps, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (N(0,1) bf16 Q/K/V)",
+            "config": {"workload": f"per-block step {args.config} (oracle, sampled heads)",
+                       "parallelism": "cpu"},
+            "cpu_baseline": cb,
+            "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default="480x480")
+    ap.add_argument("--layers", type=int, default=40)
+    ap.add_argument("--pool", type=int, default=8)
+    ap.add_argument("--cpu-heads", type=int, default=4)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        world = max(world, 1)
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+    else:
+        import torch.distributed as dist
+        if world > 1:
+            import datetime
+            import torch
+            torch.cuda.set_device(local_rank)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+        try:
+            res = run_ours(args, rank, world, local_rank)
+        finally:
+            if world > 1:
+                dist.destroy_process_group()
+    if res is not None:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,207 @@
+/*
+ * prsink.h - C ABI of the B200 (sm_100a) library for LiveAnimate's PR-Sink per-block step.
+ *
+ * Sources (web pages about arXiv 2608.11745 "LiveAnimate: Stable Long-Form Streaming Human
+ * Animation in Real-Time"), cited below by tag:
+ *   [digest]    paper.rainbus.top/paper/2608.11745 digest; paragraphs "pipeline" (with its
+ *               inference clause), "novelty" (points 2-4), "weaknesses", "reproducibility".
+ *   [explainer] papers.ananclaw.com explainer, section "Pose-Retrieval Sink Attention (PR-Sink)".
+ *   [abstract]  HF papers abstract (Chinese translation, bittide mirror).
+ *   [news]      jiazhuangai.com article, section "three key breakthroughs", item 1.
+ *
+ * Conventions shared by every call:
+ *   - All pointers except `const prsink_layout*` point to DEVICE memory owned by the caller;
+ *     the library keeps no allocation of its own.  bf16 buffers are passed as void*.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call is asynchronous
+ *     on that stream; decisions (retrieved slot, bank action) stay on the device, so a
+ *     sequence of calls needs no host synchronisation.
+ *   - Return value: PRSINK_OK (0) or a negative PRSINK_ERR_* code.  Invalid arguments are
+ *     rejected on the host before anything is launched.  No C++ exception crosses the ABI.
+ *   - Device-side waits are bounded.  A wait that runs out records PRSINK_ERR_TIMEOUT in a
+ *     device status word; prsink_sync_status() reads and clears it.
+ *
+ * Cache layout (the "slot-indexed" cache).  For one layer, K and V caches are each
+ * bf16 [H][T][d] (head-major, d contiguous).  Physical key rows are grouped in slots:
+ *   slot 0  PRSINK_SLOT_REF      L_ref = ref_frames * L_f rows      (reference image)
+ *   slot 1  PRSINK_SLOT_STATIC   L_blk rows                         (first generated block)
+ *   slot 2  PRSINK_SLOT_DYNAMIC  L_blk rows                         (pose-retrieved block)
+ *   slot 3+s ring slot s         L_blk rows each, s = 0..R-1        (rolling window)
+ * with L_f = grid_h*grid_w, L_blk = frames_per_block*L_f and T = L_ref + (2+R)*L_blk.
+ * ([explainer] slot diagram [Static][Dynamic][Rolling t-2,t-1,t]; [digest] pipeline formula
+ * puts K_ref first; [abstract] static sink = first generated block, dynamic sink = one
+ * pose-retrieved block, three-slot rolling window.)  Block b is written into ring slot b mod R.
+ *
+ * Multi-layer buffers:  cache_kv = bf16 [n_layers][2][H][T][d]   (K then V per layer)
+ *                       bank_kv  = bf16 [n_layers][M][2][H][L_blk][d]
+ */
+#ifndef PRSINK_H
+#define PRSINK_H
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define PRSINK_OK               0
+#define PRSINK_ERR_ARG         (-1)  /* null pointer, bad size, slot out of range          */
+#define PRSINK_ERR_ALIGN       (-2)  /* a pointer is not 16-byte aligned                   */
+#define PRSINK_ERR_LAUNCH      (-3)  /* CUDA error; text from prsink_last_error()          */
+#define PRSINK_ERR_TIMEOUT     (-4)  /* a bounded device wait ran out (see sync_status)    */
+#define PRSINK_ERR_UNSUPPORTED (-5)  /* valid but not supported here (e.g. head_dim 96)    */
+
+#define PRSINK_SLOT_REF     0
+#define PRSINK_SLOT_STATIC  1
+#define PRSINK_SLOT_DYNAMIC 2
+#define PRSINK_SLOT_RING0   3
+#define PRSINK_MAX_RING     8        /* ring_slots in 1..PRSINK_MAX_RING                    */
+
+#define PRSINK_FP_FRAMES    3        /* [digest] pipeline: three frames per fingerprint     */
+#define PRSINK_FP_KEYPOINTS 62       /* [digest] pipeline: 62 keypoints per frame           */
+#define PRSINK_FP_CHANNELS  3        /* x, y, confidence ([digest] novelty, point 2)        */
+#define PRSINK_FP_DIM       558      /* 3 * 62 * 3                                          */
+#define PRSINK_MAX_BANK     32       /* bank size M in 1..PRSINK_MAX_BANK (pages: M = 5)    */
+
+/* Geometry of the bounded cache and of the rotary embedding for one attention layer. */
+typedef struct prsink_layout {
+  int n_heads;           /* H (40 for the 14B DiT; 1 in the tiny check)                     */
+  int head_dim;          /* d, 64 or 128                                                    */
+  int grid_h, grid_w;    /* latent tokens per frame = grid_h*grid_w (30x30 at 480x480)     */
+  int frames_per_block;  /* B_f latent frames per block (3, [digest] reproducibility)       */
+  int ref_frames;        /* latent frames held by the ref sink (1)                         */
+  int ring_slots;        /* R, rolling-window slots (3, [explainer])                       */
+  int rope_mode;         /* 3 = 3-D RoPE over (t,h,w); 1 = 1-D over the logical token index */
+  int rope_split[3];     /* dims given to t, h, w in 3-D mode (44,42,42 for d=128); even     */
+  float rope_base;       /* RoPE base (10000)                                               */
+  long long block_index; /* b, the block being generated; fixes the ring's age order         */
+  unsigned valid_mask;   /* bit i set = slot i holds data (bit 0 ref, 1 static, 2 dynamic,
+                            3+s ring slot s); keys of other slots are ignored               */
+} prsink_layout;
+
+/* Token counts of a layout: L_f, L_blk, L_ref and T (any out pointer may be NULL).
+ * Returns PRSINK_ERR_ARG for an invalid layout. */
+int prsink_layout_tokens(const prsink_layout* layout, long long* L_f, long long* L_blk,
+                         long long* L_ref, long long* T);
+
+/* PR-Sink attention of the current block for one layer.
+ *
+ * [digest] pipeline formula: Attn(Q_b,K,V) = softmax(Q_b [K_ref; K_<b]^T / sqrt(d)) [V_ref; V_<b]
+ * over the keys the bounded cache holds; [digest] pipeline, inference clause ("RoPE follow"):
+ * keys are cached raw (pre-RoPE) and rotated at their current cache position when attended;
+ * [digest] novelty, point 4: a reused bank entry is thereby decoupled from its timestamp.
+ *
+ * Logical key order is [ref; static; dynamic; ring oldest..newest]; frames are numbered
+ * 0,1,.. in that order, so ring slot s (holding block b' = s mod R, b' in [b-R+1, b]) sits at
+ * frames ref_frames + (2 + b' - (b-R+1)) * B_f ...  A key's 3-D position is (frame, row, col)
+ * of its token; its 1-D position is frame*L_f + row*grid_w + col.  Queries sit on the newest
+ * ring slot (the current block).  RoPE: interleaved pairs (x[2j], x[2j+1]) of each axis are
+ * rotated by pos * base^(-2j/d_axis) (RoFormer); q and k are rotated, v is not.  Scale 1/sqrt(d).
+ *
+ *   q        bf16 [L_blk][H][d]   raw queries of the current block (token-major)
+ *   k_cache  bf16 [H][T][d]       raw keys, slot-indexed (see top of file)
+ *   v_cache  bf16 [H][T][d]       values, slot-indexed
+ *   out      bf16 [L_blk][H][d]   attention output (written)
+ *   lse      f32  [H][L_blk]      natural-log log-sum-exp of the scaled scores, or NULL
+ *   dyn_src  int64 scalar or NULL: if given and < 0 the dynamic slot is treated as empty
+ *            whatever valid_mask says (lets the retrieval decision stay on the device)
+ * Rows of a query with no valid key get out = 0 and lse = -inf.
+ * Errors: PRSINK_ERR_ARG (null, sizes), PRSINK_ERR_ALIGN (16 B), PRSINK_ERR_UNSUPPORTED
+ * (head_dim not 64/128, rope table too large), PRSINK_ERR_LAUNCH. */
+int prsink_attention(const prsink_layout* layout, const void* q, const void* k_cache,
+                     const void* v_cache, void* out, float* lse, const long long* dyn_src,
+                     void* stream);
+
+/* Clean KV Update / per-pass append: write one slot's raw K and V into the caches.
+ *
+ * [digest] pipeline, inference clause: KV_cache <- KV_cache U Forward(z^0_b, t=0, C) is
+ * written into the rolling window, keys raw (pre-RoPE); the ring slot of block b is b mod R;
+ * block 0's clean K/V also fills the static sink ([abstract]).
+ *
+ *   k_new, v_new  bf16 [n][H][d] token-major (as a QKV projection emits them), n = the slot's
+ *                 row count (L_ref for the ref slot, L_blk otherwise)
+ *   k_cache, v_cache  bf16 [H][T][d]; rows of slot `dest_slot` are overwritten, no other byte
+ *   dest_slot     PRSINK_SLOT_REF / _STATIC / _DYNAMIC or PRSINK_SLOT_RING0 + s
+ * Bit copy (no rounding).  Errors: PRSINK_ERR_ARG, PRSINK_ERR_ALIGN, PRSINK_ERR_LAUNCH. */
+int prsink_kv_append(const prsink_layout* layout, const void* k_new, const void* v_new,
+                     void* k_cache, void* v_cache, int dest_slot, void* stream);
+
+/* 558-d pose fingerprint of one block.
+ *
+ * [digest] pipeline, inference clause: 62 keypoints x 3 frames x 3 values, l2-normalised;
+ * [digest] novelty, point 2: confidence channel included, failed frames zero-filled.
+ *   kp        f32 [3][62][3] (x, y, conf) per frame, flattened in that order
+ *   frame_ok  u8  [3], 0 = detection failed (the frame contributes zeros)
+ *   phi       f32 [558] (written); an all-zero vector is written as zeros
+ * Norm accumulated in float64.  Errors: PRSINK_ERR_ARG, PRSINK_ERR_LAUNCH. */
+int prsink_fingerprint(const float* kp, const unsigned char* frame_ok, float* phi, void* stream);
+
+/* Pose retrieval r(b) = argmax_i phi_b . phi_i over the bank, excluding the entry of block
+ * b-1 (already in the window), and the copy of that entry's K/V into the dynamic sink.
+ *
+ * [digest] pipeline, inference clause: retrieve before generating the block, excluding b-1,
+ * copy the entry's KV into the Dynamic Sink; [digest] novelty, point 2: cosine maximisation
+ * as one dot product over l2-normalised fingerprints.
+ *
+ *   phi_b       f32 [558]          fingerprint of the incoming block
+ *   bank_phi    f32 [M][558]       bank fingerprints
+ *   bank_src    int64 [M]          source block of each entry
+ *   bank_count  int32 scalar       entries in use (0..M), slots 0..count-1
+ *   M           bank capacity (1..PRSINK_MAX_BANK)
+ *   exclude_block  b-1 (entries with this source are not eligible)
+ *   r_out       int32 scalar (written): chosen slot, ties to the lowest slot, -1 if none
+ *   score_out   f32 scalar (written) or NULL: the chosen similarity (-inf if none)
+ *   copy_out    int32 scalar (written): 1 if the dynamic sink must be (re)filled from entry
+ *               r, i.e. r >= 0 and bank_src[r] differs from the incoming *dyn_src; else 0
+ *   dyn_src     int64 scalar, in/out: source block held by the dynamic sink (-1 = empty).
+ *               On return it is bank_src[r] (or -1 when r = -1).
+ *   bank_kv, cache_kv, n_layers: optional (all NULL/0 to skip the copy).  When given, the
+ *               dynamic slot of every layer is overwritten with bank entry r iff *copy_out.
+ * Similarities are accumulated in float64.  Errors: PRSINK_ERR_ARG, _ALIGN, _LAUNCH. */
+int prsink_retrieve(const prsink_layout* layout, const float* phi_b, const float* bank_phi,
+                    const long long* bank_src, const int* bank_count, int M,
+                    long long exclude_block, int* r_out, float* score_out, int* copy_out,
+                    long long* dyn_src, const void* bank_kv, void* cache_kv, int n_layers,
+                    void* stream);
+
+/* Diversity-driven memory-bank update after block b's Clean KV Update.
+ *
+ * [digest] novelty, point 3: exhaustive replacement minimising the mean intra-bank
+ * similarity (write for coverage, read for relevance); [digest] weaknesses, point 3 and
+ * reproducibility: M = 5, written during the first 20 blocks, then frozen.
+ * For b >= write_blocks nothing changes (action -1).  While count < M the block is inserted
+ * at slot count.  Otherwise the options "keep" and "replace slot j" are scored by the mean
+ * of phi_i . phi_j over unordered pairs of the resulting bank (float64); the least wins,
+ * ties go to keep, then to the lowest j.
+ *
+ *   bank_phi   f32 [M][558]  in/out      bank_src  int64 [M] in/out      bank_count int32 in/out
+ *   phi_b      f32 [558]     fingerprint of block b
+ *   action_out int32 scalar (written): slot written, or -1
+ *   cache_kv, bank_kv, n_layers: optional (NULL/0 to skip).  When given and action >= 0, the
+ *               clean K/V of block b (ring slot b mod R of every layer) is copied into bank
+ *               entry `action`.
+ * Errors: PRSINK_ERR_ARG, PRSINK_ERR_ALIGN, PRSINK_ERR_LAUNCH. */
+int prsink_bank_update(const prsink_layout* layout, float* bank_phi, long long* bank_src,
+                       int* bank_count, int M, const float* phi_b, long long b,
+                       int write_blocks, int* action_out, const void* cache_kv, void* bank_kv,
+                       int n_layers, void* stream);
+
+/* Synchronise `stream`, then read and clear the device status word: PRSINK_OK, or
+ * PRSINK_ERR_TIMEOUT if a bounded wait ran out since the last call, or PRSINK_ERR_LAUNCH. */
+int prsink_sync_status(void* stream);
+
+/* Text of the last host-side error of this thread ("" if none).  Owned by the library. */
+const char* prsink_last_error(void);
+
+/* Number of kernels this library launched since load (host counter). */
+long long prsink_launch_count(void);
+
+/* Self-test of the bounded-wait path: launches one block that waits on a barrier nothing
+ * signals, gives up after `timeout_ns` (clamped to [1e3, 5e9] ns), records
+ * PRSINK_ERR_TIMEOUT in the status word and returns.  No GPU fault, no hang. */
+int prsink_debug_wait_timeout(long long timeout_ns, void* stream);
+
+/* Library ABI version (increments on any signature change). */
+int prsink_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* PRSINK_H */

@@ -1,0 +1,652 @@
+// PR-Sink attention for sm_100a: TMA-staged K/V tiles from the slot-indexed cache, RoPE of the
+// raw keys fused between the TMA landing and the tensor-core read ("RoPE follow"), tcgen05 MMAs
+// with accumulators in tensor memory, fp32 online softmax, no materialised score matrix.
+//
+// One CTA computes one 128-query tile of one head.  Warp roles (320 threads):
+//   warps 0-3  softmax: thread t owns query row t (= TMEM lane t); reads S from TMEM, keeps
+//              the running max / sum, writes P (bf16) to shared memory, rescales O in TMEM
+//              when the max grows by more than 2^8, and finally normalises and stores O;
+//   warp  4    TMA producer: Q once, then K and V tiles into a 2-stage ring;
+//   warp  5    MMA issuer: S = Q K^T into one of two TMEM score buffers, O += P V;
+//   warps 6-9  rotation: rotate Q once and every K tile in place at the keys' current
+//              logical positions (interleaved RoFormer pairs, per-axis tables in shared
+//              memory), zero the rows of empty slots, and hand the tile to the MMA warp.
+// Key tiles run over the physical rows of the cache; softmax attention does not depend on the
+// order of the keys, only on their positions, so each key is rotated at the position of its
+// logical slot and no gather is needed.  Tiles inside empty slots are skipped.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include <cmath>
+#include <mutex>
+
+#include "prsink_internal.cuh"
+
+namespace prsink {
+namespace attn {
+
+constexpr int BM = 128;                 // queries per CTA
+constexpr int BN = 128;                 // keys per tile
+constexpr int kThreads = 320;
+constexpr int kProducerWarp = 4;
+constexpr int kMmaWarp = 5;
+constexpr int kRotWarp0 = 6;
+constexpr int kMaxSlots = 3 + PRSINK_MAX_RING;
+constexpr uint32_t kTmemCols = 512;
+constexpr int kTableMaxBytes = 32 * 1024;
+constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale O when the max grows > 2^8
+
+struct Params {
+  int H, L_blk, T, L_f, grid_h, grid_w;
+  int n_slots;
+  int slot_start[kMaxSlots + 1];
+  int slot_frame[kMaxSlots];
+  unsigned valid_mask;
+  int q_frame;                          // logical frame of the current block's first frame
+  int rope_mode;                        // 1 or 3
+  int rd[3];                            // rotated pairs per axis (1-D: D/2, 0, 0)
+  int n_frames;                         // frames of the logical layout
+  int tab_h_off, tab_w_off, tab_entries;  // float2 offsets of the tables
+  double log2_base;
+  float scale_log2;                     // log2(e) / sqrt(d)
+  __nv_bfloat16* out;
+  float* lse;
+  const long long* dyn_src;
+  int* status;
+  unsigned long long timeout_ns;
+};
+
+enum Bar {
+  B_QFULL = 0, B_QREADY = 1, B_KVFULL = 2, B_KREADY = 4, B_KVEMPTY = 6, B_SFULL = 8,
+  B_SFREE = 10, B_PFULL = 12, B_ODONE = 13, B_FINAL = 14, B_COUNT = 15
+};
+
+template <int D>
+struct Layout {
+  static constexpr int kPanels = D / 64;
+  static constexpr int kPanelBytes = 128 * 128;          // 128 rows x 128 B (64 bf16)
+  static constexpr int kTileBytes = kPanels * kPanelBytes;
+  static constexpr int kQ = 0;
+  static constexpr int kK = kQ + kTileBytes;             // 2 stages
+  static constexpr int kV = kK + 2 * kTileBytes;         // 2 stages
+  static constexpr int kP = kV + 2 * kTileBytes;         // 128 x 128 bf16, 2 panels
+  static constexpr int kTab = kP + 2 * kPanelBytes;
+  static constexpr uint32_t kIdescS = idesc_bf16_f32(128, BN, false, false);
+  static constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, false, true);
+};
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ bool tile_live(int n, unsigned vm, const Params& p) {
+  const int lo = n * BN, hi = min(lo + BN, p.T);
+  for (int s = 0; s < p.n_slots; ++s)
+    if (((vm >> s) & 1u) && p.slot_start[s] < hi && p.slot_start[s + 1] > lo) return true;
+  return false;
+}
+
+__device__ __forceinline__ bool tile_full(int n, unsigned vm, const Params& p) {
+  const int lo = n * BN, hi = lo + BN;
+  if (hi > p.T) return false;
+  for (int s = 0; s < p.n_slots; ++s)
+    if (!((vm >> s) & 1u) && p.slot_start[s] < hi && p.slot_start[s + 1] > lo) return false;
+  return true;
+}
+
+__device__ __forceinline__ int slot_of(int row, const Params& p) {
+  int s = 0;
+  while (s + 1 < p.n_slots && row >= p.slot_start[s + 1]) ++s;
+  return s;
+}
+
+// Bounded wait that ignores the abort flag (used while draining after an abort).
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64_t ns) {
+  const uint64_t dl = globaltimer() + ns;
+  while (!mbar_try_wait(bar, parity))
+    if (globaltimer() > dl) break;
+}
+
+// Rotate one 128-byte-swizzled row (D bf16 over D/64 panels) in place at position
+// (frame, tok); or zero it when `zero` is set.
+template <int D>
+__device__ __forceinline__ void rotate_row(uint8_t* tile, int r, int frame, int tok, bool zero,
+                                           const float2* __restrict__ tab, const Params& p) {
+  const int y = tok / p.grid_w, x = tok - (tok / p.grid_w) * p.grid_w;
+  const float2* rowT;
+  const float2* rowH;
+  const float2* rowW;
+  if (p.rope_mode == 3) {
+    rowT = tab + frame * p.rd[0];
+    rowH = tab + p.tab_h_off + y * p.rd[1];
+    rowW = tab + p.tab_w_off + x * p.rd[2];
+  } else {
+    rowT = tab + frame * (D / 2);                  // angle of frame*L_f
+    rowH = tab + p.tab_h_off + tok * (D / 2);      // angle of the in-frame token index
+    rowW = nullptr;
+  }
+  const int r0 = p.rd[0], r01 = p.rd[0] + p.rd[1];
+#pragma unroll
+  for (int pp = 0; pp < D / 64; ++pp) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      uint4* ptr = reinterpret_cast<uint4*>(tile + pp * 16384 + r * 128 + ((c ^ (r & 7)) << 4));
+      if (zero) {
+        *ptr = make_uint4(0, 0, 0, 0);
+        continue;
+      }
+      uint4 v = *ptr;
+      uint32_t* w = reinterpret_cast<uint32_t*>(&v);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int P = pp * 32 + c * 4 + i;
+        float2 cs;
+        if (p.rope_mode == 3) {
+          cs = P < r0 ? rowT[P] : (P < r01 ? rowH[P - r0] : rowW[P - r01]);
+        } else {
+          const float2 a = rowT[P], b = rowH[P];
+          cs = make_float2(a.x * b.x - a.y * b.y, a.y * b.x + a.x * b.y);
+        }
+        __nv_bfloat162 pr = *reinterpret_cast<__nv_bfloat162*>(&w[i]);
+        const float x0 = __low2float(pr), x1 = __high2float(pr);
+        const float y0 = x0 * cs.x - x1 * cs.y;
+        const float y1 = x0 * cs.y + x1 * cs.x;
+        pr = __floats2bfloat162_rn(y0, y1);
+        w[i] = *reinterpret_cast<uint32_t*>(&pr);
+      }
+      *ptr = v;
+    }
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
+                        const __grid_constant__ CUtensorMap tm_k,
+                        const __grid_constant__ CUtensorMap tm_v, const Params p) {
+  using LY = Layout<D>;
+  extern __shared__ uint8_t dsmem[];
+  __shared__ __align__(8) uint64_t bars[B_COUNT];
+  __shared__ uint32_t tmem_base_s;
+  __shared__ AbortState ab;
+  __shared__ unsigned vmask_s;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t raw = smem_u32(dsmem);
+  const uint32_t sb = (raw + 1023u) & ~1023u;            // 1 KB aligned base (swizzle atoms)
+  uint8_t* gb = dsmem + (sb - raw);
+  const uint32_t sQ = sb + LY::kQ, sK = sb + LY::kK, sV = sb + LY::kV, sP = sb + LY::kP;
+  float2* tab = reinterpret_cast<float2*>(gb + LY::kTab);
+  auto bar = [&](int i) { return smem_u32(&bars[i]); };
+
+  const int q0 = blockIdx.x * BM;
+  const int h = blockIdx.y;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(B_QFULL), 1);
+    mbar_init(bar(B_QREADY), 128);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(B_KVFULL + s), 1);
+      mbar_init(bar(B_KREADY + s), 128);
+      mbar_init(bar(B_KVEMPTY + s), 1);
+      mbar_init(bar(B_SFULL + s), 1);
+      mbar_init(bar(B_SFREE + s), 128);
+    }
+    mbar_init(bar(B_PFULL), 128);
+    mbar_init(bar(B_ODONE), 1);
+    mbar_init(bar(B_FINAL), 1);
+    ab.flag = 0;
+    unsigned vm = p.valid_mask;
+    if (p.dyn_src && *p.dyn_src < 0) vm &= ~(1u << PRSINK_SLOT_DYNAMIC);
+    vmask_s = vm;
+    fence_barrier_init();
+  }
+  if (warp == kProducerWarp && lane == 0) {
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(smem_u32(&tmem_base_s), kTmemCols);
+    tmem_relinquish();
+  }
+  // RoPE tables: cos/sin of pos * base^(-2j/d_axis), computed in double, stored as float2.
+  for (int e = threadIdx.x; e < p.tab_entries; e += kThreads) {
+    int pos, j, da;
+    if (p.rope_mode == 3) {
+      if (e < p.tab_h_off) { pos = e / p.rd[0]; j = e % p.rd[0]; da = 2 * p.rd[0]; }
+      else if (e < p.tab_w_off) { const int f = e - p.tab_h_off; pos = f / p.rd[1]; j = f % p.rd[1]; da = 2 * p.rd[1]; }
+      else { const int f = e - p.tab_w_off; pos = f / p.rd[2]; j = f % p.rd[2]; da = 2 * p.rd[2]; }
+    } else {
+      da = D;
+      if (e < p.tab_h_off) { pos = (e / (D / 2)) * p.L_f; j = e % (D / 2); }
+      else { const int f = e - p.tab_h_off; pos = f / (D / 2); j = f % (D / 2); }
+    }
+    const double theta = exp2(-(2.0 * j / da) * p.log2_base);
+    double sn, cs;
+    sincos(static_cast<double>(pos) * theta, &sn, &cs);
+    tab[e] = make_float2(static_cast<float>(cs), static_cast<float>(sn));
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  const uint32_t tmem = tmem_base_s;
+  const unsigned vm = vmask_s;
+  const uint64_t deadline = globaltimer() + p.timeout_ns;
+  const int n_tiles = (p.T + BN - 1) / BN;
+
+  if (warp == kProducerWarp) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      mbar_arrive_expect_tx(bar(B_QFULL), LY::kTileBytes);
+      for (int pp = 0; pp < D / 64; ++pp)
+        tma_load_3d(sQ + pp * 16384, &tm_q, bar(B_QFULL), pp * 64, h, q0);
+      int it = 0;
+      int issued[2] = {-1, -1};
+      for (int n = 0; n < n_tiles; ++n) {
+        if (!tile_live(n, vm, p)) continue;
+        const int st = it & 1;
+        if (it >= 2 && !mbar_wait(bar(B_KVEMPTY + st), ((it >> 1) - 1) & 1, &ab, deadline, p.status))
+          break;
+        mbar_arrive_expect_tx(bar(B_KVFULL + st), 2 * LY::kTileBytes);
+        for (int pp = 0; pp < D / 64; ++pp) {
+          tma_load_3d(sK + st * LY::kTileBytes + pp * 16384, &tm_k, bar(B_KVFULL + st), pp * 64,
+                      n * BN, h);
+          tma_load_3d(sV + st * LY::kTileBytes + pp * 16384, &tm_v, bar(B_KVFULL + st), pp * 64,
+                      n * BN, h);
+        }
+        issued[st] = it;
+        ++it;
+      }
+      if (ab.flag) {     // let copies in flight land before the CTA's shared memory goes away
+        drain_wait(bar(B_QFULL), 0, 100000000ull);
+        for (int s = 0; s < 2; ++s)
+          if (issued[s] >= 0) drain_wait(bar(B_KVFULL + s), (issued[s] >> 1) & 1, 100000000ull);
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      bool ok = mbar_wait(bar(B_QREADY), 0, &ab, deadline, p.status);
+      tc_fence_after();
+      const uint32_t tO = tmem + 256;
+      auto issue_pv = [&](int j) -> bool {
+        if (!mbar_wait(bar(B_PFULL), j & 1, &ab, deadline, p.status)) return false;
+        tc_fence_after();
+        const uint32_t v_base = sV + (j & 1) * LY::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          const uint64_t a = sdesc_sw128(sP + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+          const uint64_t b = sdesc_sw128(v_base + kk * 2048, 16384, 1024);
+          umma_ss(tO, a, b, LY::kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(bar(B_ODONE));
+        umma_commit(bar(B_KVEMPTY + (j & 1)));
+        return true;
+      };
+      int it = 0;
+      for (int n = 0; ok && n < n_tiles; ++n) {
+        if (!tile_live(n, vm, p)) continue;
+        const int st = it & 1;
+        if (!mbar_wait(bar(B_KREADY + st), (it >> 1) & 1, &ab, deadline, p.status)) { ok = false; break; }
+        if (it >= 2 && !mbar_wait(bar(B_SFREE + st), ((it >> 1) - 1) & 1, &ab, deadline, p.status)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t tS = tmem + st * 128;
+        const uint32_t k_base = sK + st * LY::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t a = sdesc_sw128(sQ + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+          const uint64_t b = sdesc_sw128(k_base + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+          umma_ss(tS, a, b, LY::kIdescS, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(bar(B_SFULL + st));
+        if (it >= 1 && !issue_pv(it - 1)) { ok = false; break; }
+        ++it;
+      }
+      if (ok && it >= 1) issue_pv(it - 1);
+      if (ab.flag) {     // wait for every MMA issued so far before TMEM is released
+        umma_commit(bar(B_FINAL));
+        drain_wait(bar(B_FINAL), 0, 100000000ull);
+      }
+    }
+  } else if (warp >= kRotWarp0) {
+    // ------------------------------------------------------------------ rotation
+    const int rt = threadIdx.x - kRotWarp0 * 32;          // row of the tile, 0..127
+    if (mbar_wait(bar(B_QFULL), 0, &ab, deadline, p.status)) {
+      const int qi = q0 + rt;
+      if (qi < p.L_blk)
+        rotate_row<D>(gb + LY::kQ, rt, p.q_frame + qi / p.L_f, qi % p.L_f, false, tab, p);
+      fence_proxy_async_smem();
+      mbar_arrive(bar(B_QREADY));
+      int it = 0;
+      for (int n = 0; n < n_tiles; ++n) {
+        if (!tile_live(n, vm, p)) continue;
+        const int st = it & 1;
+        if (!mbar_wait(bar(B_KVFULL + st), (it >> 1) & 1, &ab, deadline, p.status)) break;
+        const int row = n * BN + rt;
+        if (row < p.T) {
+          const int s = slot_of(row, p);
+          const int u = row - p.slot_start[s];
+          const bool empty = !((vm >> s) & 1u);
+          uint8_t* kt = gb + LY::kK + st * LY::kTileBytes;
+          rotate_row<D>(kt, rt, p.slot_frame[s] + u / p.L_f, u % p.L_f, empty, tab, p);
+          if (empty) rotate_row<D>(gb + LY::kV + st * LY::kTileBytes, rt, 0, 0, true, tab, p);
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(bar(B_KREADY + st));
+        ++it;
+      }
+    }
+  } else {
+    // ------------------------------------------------------------------ softmax (warps 0-3)
+    const int t = threadIdx.x;                            // query row = TMEM lane
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t tO = tmem + lane_off + 256;
+    float m = -INFINITY, l = 0.f;
+    int it = 0;
+    bool ok = true;
+    uint8_t* prow = gb + LY::kP;
+    for (int n = 0; n < n_tiles; ++n) {
+      if (!tile_live(n, vm, p)) continue;
+      const int st = it & 1;
+      ok = mbar_wait(bar(B_SFULL + st), (it >> 1) & 1, &ab, deadline, p.status);
+      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }   // tcgen05.ld is warp-collective
+      tc_fence_after();
+      uint32_t s[128];
+      const uint32_t tS = tmem + lane_off + st * 128;
+      tmem_ld32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
+      tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
+      tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
+      tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(bar(B_SFREE + st));
+      float x[128];
+#pragma unroll
+      for (int c = 0; c < 128; ++c) x[c] = __uint_as_float(s[c]) * p.scale_log2;
+      if (!tile_full(n, vm, p)) {
+        // columns of empty slots and past the end of the cache: 4 mask words, built per slot
+        const int lo = n * BN;
+        uint32_t mw[4] = {~0u, ~0u, ~0u, ~0u};
+        for (int s2 = 0; s2 <= p.n_slots; ++s2) {
+          int a, e;
+          if (s2 < p.n_slots) {
+            if ((vm >> s2) & 1u) continue;
+            a = p.slot_start[s2] - lo;
+            e = p.slot_start[s2 + 1] - lo;
+          } else {
+            a = p.T - lo;
+            e = BN;
+          }
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            const int cl = max(a, w * 32), ch = min(e, w * 32 + 32);
+            if (cl < ch) {
+              const uint32_t bits = (ch - cl == 32) ? ~0u : (((1u << (ch - cl)) - 1u) << (cl - w * 32));
+              mw[w] &= ~bits;
+            }
+          }
+        }
+#pragma unroll
+        for (int c = 0; c < 128; ++c)
+          if (!((mw[c >> 5] >> (c & 31)) & 1u)) x[c] = -INFINITY;
+      }
+      float mt = x[0];
+#pragma unroll
+      for (int c = 1; c < 128; ++c) mt = fmaxf(mt, x[c]);
+      float alpha = 1.f;
+      bool rescale = false;
+      if (it == 0) {
+        m = mt;
+      } else if (mt > m + kRescaleThreshold) {
+        alpha = ex2(m - mt);
+        m = mt;
+        rescale = true;
+      }
+      float sum = 0.f;
+      uint32_t pk[64];                          // P as bf16 pairs: keeps the rescale in registers
+#pragma unroll
+      for (int c = 0; c < 128; c += 2) {
+        const float p0 = ex2(x[c] - m), p1 = ex2(x[c + 1] - m);
+        sum += p0 + p1;
+        __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
+        pk[c >> 1] = *reinterpret_cast<uint32_t*>(&b2);
+      }
+      l = l * alpha + sum;
+      if (it >= 1) {
+        ok = mbar_wait(bar(B_ODONE), (it - 1) & 1, &ab, deadline, p.status);
+        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+        tc_fence_after();
+      }
+      if (__any_sync(0xffffffffu, rescale)) {   // rows that keep their max scale by alpha = 1
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t o[32];
+          tmem_ld32(tO + cc * 32, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32(tO + cc * 32, o);
+        }
+        tmem_wait_st();
+      }
+#pragma unroll
+      for (int pp = 0; pp < 2; ++pp) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const int k = pp * 32 + c * 4;
+          *reinterpret_cast<uint4*>(prow + pp * 16384 + t * 128 + ((c ^ (t & 7)) << 4)) =
+              make_uint4(pk[k], pk[k + 1], pk[k + 2], pk[k + 3]);
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(bar(B_PFULL));
+      ++it;
+    }
+    // epilogue: O / l -> bf16, one 2*D-byte row per thread
+    const int qi = q0 + t;
+    float inv = 0.f;
+    bool have = false;
+    if (__all_sync(0xffffffffu, ok) && it > 0) {
+      have = mbar_wait(bar(B_ODONE), (it - 1) & 1, &ab, deadline, p.status);
+      have = __all_sync(0xffffffffu, have);
+      tc_fence_after();
+      inv = l > 0.f ? 1.f / l : 0.f;
+    }
+    __nv_bfloat16* orow = p.out + (static_cast<size_t>(qi) * p.H + h) * D;
+#pragma unroll
+    for (int cc = 0; cc < D / 32; ++cc) {
+      uint32_t o[32];
+      if (have) {                     // warp-uniform
+        tmem_ld32(tO + cc * 32, o);
+        tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[i] = 0u;
+      }
+      if (qi < p.L_blk) {
+#pragma unroll
+        for (int i = 0; i < 32; i += 8) {
+          __nv_bfloat162 b0 = __floats2bfloat162_rn(__uint_as_float(o[i + 0]) * inv, __uint_as_float(o[i + 1]) * inv);
+          __nv_bfloat162 b1 = __floats2bfloat162_rn(__uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
+          __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(o[i + 4]) * inv, __uint_as_float(o[i + 5]) * inv);
+          __nv_bfloat162 b3 = __floats2bfloat162_rn(__uint_as_float(o[i + 6]) * inv, __uint_as_float(o[i + 7]) * inv);
+          uint4 v;
+          v.x = *reinterpret_cast<uint32_t*>(&b0);
+          v.y = *reinterpret_cast<uint32_t*>(&b1);
+          v.z = *reinterpret_cast<uint32_t*>(&b2);
+          v.w = *reinterpret_cast<uint32_t*>(&b3);
+          *reinterpret_cast<uint4*>(orow + cc * 32 + i) = v;
+        }
+      }
+    }
+    if (p.lse && qi < p.L_blk)
+      p.lse[static_cast<size_t>(h) * p.L_blk + qi] =
+          have ? (m + log2f(l)) * 0.69314718055994530942f : -INFINITY;
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------- host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess && q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// 3-D bf16 tensor map with a 64 x box1 x box2 box and 128-byte swizzle.
+static int make_map(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                    uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box1,
+                    uint32_t box2) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) {
+    set_error("cuTensorMapEncodeTiled is not available from the driver");
+    return PRSINK_ERR_LAUNCH;
+  }
+  const cuuint64_t dims[3] = {d0, d1, d2};
+  const cuuint64_t strides[2] = {stride1_bytes, stride2_bytes};
+  const cuuint32_t box[3] = {64, box1, box2};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    set_error("cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+    return PRSINK_ERR_LAUNCH;
+  }
+  return PRSINK_OK;
+}
+
+template <int D>
+static int launch(const prsink_layout* L, const Geometry& g, const void* q, const void* k,
+                  const void* v, Params& p, cudaStream_t st) {
+  CUtensorMap mq, mk, mv;
+  int rc = make_map(&mq, q, D, L->n_heads, g.L_blk, 2ull * D, 2ull * D * L->n_heads, 1, BM);
+  if (!rc) rc = make_map(&mk, k, D, g.T, L->n_heads, 2ull * D, 2ull * D * g.T, BN, 1);
+  if (!rc) rc = make_map(&mv, v, D, g.T, L->n_heads, 2ull * D, 2ull * D * g.T, BN, 1);
+  if (rc) return rc;
+  const int tab_bytes = p.tab_entries * 8;
+  int smem = Layout<D>::kTab + tab_bytes + 1024;
+  if (smem < 120 * 1024) smem = 120 * 1024;     // one CTA per SM (it holds all 512 TMEM columns)
+  static int attr_bytes[64] = {0};      // largest size already allowed, per device
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  if (attr_bytes[dev] < smem) {
+    if (cudaFuncSetAttribute(prsink_attention_kernel<D>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return check_launch("prsink_attention: shared memory attribute");
+    attr_bytes[dev] = smem;
+  }
+  dim3 grid((g.L_blk + BM - 1) / BM, L->n_heads);
+  prsink_attention_kernel<D><<<grid, kThreads, smem, st>>>(mq, mk, mv, p);
+  count_launch();
+  return check_launch("prsink_attention");
+}
+
+}  // namespace attn
+}  // namespace prsink
+
+using namespace prsink;
+
+extern "C" int prsink_attention(const prsink_layout* layout, const void* q, const void* k_cache,
+                                const void* v_cache, void* out, float* lse,
+                                const long long* dyn_src, void* stream) {
+  using namespace prsink::attn;
+  Geometry g;
+  int rc = geometry(layout, &g);
+  if (rc) return rc;
+  if (!q || !k_cache || !v_cache || !out) {
+    set_error("prsink_attention: null pointer");
+    return PRSINK_ERR_ARG;
+  }
+  const int D = layout->head_dim;
+  if (D != 64 && D != 128) {
+    set_error("prsink_attention: head_dim %d not supported (64 or 128)", D);
+    return PRSINK_ERR_UNSUPPORTED;
+  }
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
+      (lse && (reinterpret_cast<uintptr_t>(lse) & 3u))) {
+    set_error("prsink_attention: q, k_cache, v_cache, out must be 16-byte aligned");
+    return PRSINK_ERR_ALIGN;
+  }
+  Params p{};
+  p.H = layout->n_heads;
+  p.L_blk = static_cast<int>(g.L_blk);
+  p.T = static_cast<int>(g.T);
+  p.L_f = static_cast<int>(g.L_f);
+  p.grid_h = layout->grid_h;
+  p.grid_w = layout->grid_w;
+  p.n_slots = g.n_slots;
+  for (int s = 0; s <= g.n_slots; ++s) p.slot_start[s] = static_cast<int>(g.slot_start[s]);
+  const int R = layout->ring_slots;
+  const int Bf = layout->frames_per_block;
+  const long long b = layout->block_index;
+  p.slot_frame[PRSINK_SLOT_REF] = 0;
+  p.slot_frame[PRSINK_SLOT_STATIC] = layout->ref_frames;
+  p.slot_frame[PRSINK_SLOT_DYNAMIC] = layout->ref_frames + Bf;
+  for (int s = 0; s < R; ++s) {
+    // ring slot s holds block b' = s (mod R), b' in [b-R+1, b]; its age rank is b'-(b-R+1)
+    const long long oldest = b - R + 1;
+    const int rank = static_cast<int>((((s - oldest) % R) + R) % R);
+    p.slot_frame[PRSINK_SLOT_RING0 + s] = layout->ref_frames + (2 + rank) * Bf;
+  }
+  p.q_frame = layout->ref_frames + (2 + R - 1) * Bf;
+  p.n_frames = layout->ref_frames + (2 + R) * Bf;
+  p.valid_mask = layout->valid_mask & ((1u << g.n_slots) - 1u);
+  p.rope_mode = layout->rope_mode;
+  if (p.rope_mode == 3) {
+    p.rd[0] = layout->rope_split[0] / 2;
+    p.rd[1] = layout->rope_split[1] / 2;
+    p.rd[2] = layout->rope_split[2] / 2;
+    p.tab_h_off = p.n_frames * p.rd[0];
+    p.tab_w_off = p.tab_h_off + layout->grid_h * p.rd[1];
+    p.tab_entries = p.tab_w_off + layout->grid_w * p.rd[2];
+  } else {
+    p.rd[0] = D / 2;
+    p.rd[1] = 0;
+    p.rd[2] = 0;
+    p.tab_h_off = p.n_frames * (D / 2);
+    p.tab_w_off = p.tab_h_off + p.L_f * (D / 2);
+    p.tab_entries = p.tab_w_off;
+  }
+  if (p.tab_entries * 8 > kTableMaxBytes) {
+    set_error("prsink_attention: RoPE tables need %d bytes of shared memory (max %d)",
+              p.tab_entries * 8, kTableMaxBytes);
+    return PRSINK_ERR_UNSUPPORTED;
+  }
+  p.log2_base = std::log2(static_cast<double>(layout->rope_base));
+  p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.dyn_src = dyn_src;
+  p.status = status_word_ptr();
+  p.timeout_ns = 2000000000ull;
+  if (!p.status) return PRSINK_ERR_LAUNCH;
+  if (g.L_blk == 0) return PRSINK_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return D == 128 ? launch<128>(layout, g, q, k_cache, v_cache, p, st)
+                  : launch<64>(layout, g, q, k_cache, v_cache, p, st);
+}

@@ -1,0 +1,186 @@
+// KV cache writes of the PR-Sink step, all plain HBM-bound byte copies:
+//   * prsink_kv_append: a block's raw K/V, token-major [n][H][d] as a QKV projection emits
+//     them, into one slot of the head-major caches [H][T][d] (a transpose at 2*d-byte rows);
+//   * the dynamic-sink fill (bank entry r -> dynamic slot of every layer) and the bank store
+//     (ring slot of block b -> bank entry `action` of every layer), both predicated on a
+//     decision that stays in device memory.
+// Every thread moves 16-byte chunks; a 256-byte head row is one 16-lane run, so reads and
+// writes are fully coalesced without staging through shared memory.
+#include "prsink_internal.cuh"
+
+namespace prsink {
+
+constexpr int kCopyThreads = 256;
+constexpr int kCopyUnroll = 4;
+
+// k_new/v_new [n][H][C] 16-byte chunks -> cache [H][T][C] rows start..start+n.
+__global__ void __launch_bounds__(kCopyThreads)
+append_kernel(const uint4* __restrict__ k_new, const uint4* __restrict__ v_new,
+              uint4* __restrict__ k_cache, uint4* __restrict__ v_cache, uint32_t n_chunks,
+              uint32_t H, uint32_t C, uint64_t T, uint64_t start) {
+  const uint4* __restrict__ src = blockIdx.y ? v_new : k_new;
+  uint4* __restrict__ dst = blockIdx.y ? v_cache : k_cache;
+  const uint32_t HC = H * C;
+  const uint32_t stride = gridDim.x * kCopyThreads * kCopyUnroll;
+  for (uint32_t base = blockIdx.x * kCopyThreads * kCopyUnroll + threadIdx.x; base < n_chunks;
+       base += stride) {
+    uint4 v[kCopyUnroll];
+#pragma unroll
+    for (int u = 0; u < kCopyUnroll; ++u) {
+      const uint32_t i = base + u * kCopyThreads;
+      if (i < n_chunks) v[u] = __ldcs(src + i);
+    }
+#pragma unroll
+    for (int u = 0; u < kCopyUnroll; ++u) {
+      const uint32_t i = base + u * kCopyThreads;
+      if (i < n_chunks) {
+        const uint32_t tok = i / HC;
+        const uint32_t rem = i - tok * HC;
+        const uint32_t h = rem / C;
+        const uint32_t c = rem - h * C;
+        dst[(static_cast<uint64_t>(h) * T + start + tok) * C + c] = v[u];
+      }
+    }
+  }
+}
+
+// Segment copy: segment y (one (layer, k|v, head) run of `seg_chunks` contiguous chunks) from
+// src + y-dependent offset to dst + y-dependent offset.  Runs only if *flag != 0 (flag may be
+// null) and *sel >= 0; *sel picks the bank entry on the bank side.
+struct SegCopy {
+  const uint4* src;
+  uint4* dst;
+  uint64_t seg_chunks;          // chunks per (layer, kv, head) run
+  uint32_t H;
+  // chunk offsets: offset = layer*L + kv*KV + head*HD (+ sel*SEL on the bank side)
+  uint64_t src_layer, src_kv, src_head, src_sel, src_base;
+  uint64_t dst_layer, dst_kv, dst_head, dst_sel, dst_base;
+};
+
+__global__ void __launch_bounds__(kCopyThreads)
+seg_copy_kernel(SegCopy p, const int* __restrict__ sel, const int* __restrict__ flag) {
+  const int s = *sel;
+  if (s < 0 || (flag && *flag == 0)) return;
+  const uint32_t y = blockIdx.y;               // = (layer*2 + kv)*H + head
+  const uint32_t head = y % p.H;
+  const uint32_t lk = y / p.H;
+  const uint32_t kv = lk & 1u;
+  const uint32_t layer = lk >> 1;
+  const uint4* __restrict__ src = p.src + p.src_base + layer * p.src_layer + kv * p.src_kv +
+                                  head * p.src_head + static_cast<uint64_t>(s) * p.src_sel;
+  uint4* __restrict__ dst = p.dst + p.dst_base + layer * p.dst_layer + kv * p.dst_kv +
+                            head * p.dst_head + static_cast<uint64_t>(s) * p.dst_sel;
+  const uint64_t stride = static_cast<uint64_t>(gridDim.x) * kCopyThreads * kCopyUnroll;
+  for (uint64_t base = static_cast<uint64_t>(blockIdx.x) * kCopyThreads * kCopyUnroll +
+                       threadIdx.x;
+       base < p.seg_chunks; base += stride) {
+    uint4 v[kCopyUnroll];
+#pragma unroll
+    for (int u = 0; u < kCopyUnroll; ++u) {
+      const uint64_t i = base + u * kCopyThreads;
+      if (i < p.seg_chunks) v[u] = __ldcs(src + i);
+    }
+#pragma unroll
+    for (int u = 0; u < kCopyUnroll; ++u) {
+      const uint64_t i = base + u * kCopyThreads;
+      if (i < p.seg_chunks) dst[i] = v[u];
+    }
+  }
+}
+
+static int grid_for(uint64_t chunks) {
+  uint64_t g = (chunks + kCopyThreads * kCopyUnroll - 1) / (kCopyThreads * kCopyUnroll);
+  if (g < 1) g = 1;
+  if (g > 148ull * 16) g = 148ull * 16;
+  return static_cast<int>(g);
+}
+
+// Launch the predicated copy between bank entry *sel and cache slot `slot` of every layer.
+// to_cache = true: bank -> cache (dynamic-sink fill); false: cache -> bank (bank store).
+int launch_bank_cache_copy(const prsink_layout* L, const Geometry& g, int M, int n_layers,
+                           const void* bank_kv, const void* cache_kv, bool to_cache, int slot,
+                           const int* sel, const int* flag, cudaStream_t st) {
+  const uint64_t C = static_cast<uint64_t>(L->head_dim) * 2 / 16;   // chunks per row
+  const uint64_t H = L->n_heads;
+  // cache_kv [layers][2][H][T][d]; bank_kv [layers][M][2][H][L_blk][d]
+  const uint64_t cache_head = static_cast<uint64_t>(g.T) * C;
+  const uint64_t cache_kv_s = H * cache_head;
+  const uint64_t cache_layer = 2 * cache_kv_s;
+  const uint64_t bank_head = static_cast<uint64_t>(g.L_blk) * C;
+  const uint64_t bank_kv_s = H * bank_head;
+  const uint64_t bank_sel = 2 * bank_kv_s;
+  const uint64_t bank_layer = static_cast<uint64_t>(M) * bank_sel;
+  const uint64_t slot_off = static_cast<uint64_t>(g.slot_start[slot]) * C;
+  SegCopy p{};
+  p.seg_chunks = bank_head;
+  p.H = static_cast<uint32_t>(H);
+  if (to_cache) {
+    p.src = static_cast<const uint4*>(bank_kv);
+    p.dst = static_cast<uint4*>(const_cast<void*>(cache_kv));
+    p.src_layer = bank_layer; p.src_kv = bank_kv_s; p.src_head = bank_head; p.src_sel = bank_sel;
+    p.src_base = 0;
+    p.dst_layer = cache_layer; p.dst_kv = cache_kv_s; p.dst_head = cache_head; p.dst_sel = 0;
+    p.dst_base = slot_off;
+  } else {
+    p.src = static_cast<const uint4*>(cache_kv);
+    p.dst = static_cast<uint4*>(const_cast<void*>(bank_kv));
+    p.src_layer = cache_layer; p.src_kv = cache_kv_s; p.src_head = cache_head; p.src_sel = 0;
+    p.src_base = slot_off;
+    p.dst_layer = bank_layer; p.dst_kv = bank_kv_s; p.dst_head = bank_head; p.dst_sel = bank_sel;
+    p.dst_base = 0;
+  }
+  const uint64_t segs = static_cast<uint64_t>(n_layers) * 2 * H;
+  if (segs > 65535) {
+    set_error("too many (layer, k/v, head) segments: %llu", (unsigned long long)segs);
+    return PRSINK_ERR_ARG;
+  }
+  // enough CTAs in flight for HBM: about 4 per SM over all segments
+  uint64_t gx = (148ull * 4 + segs - 1) / segs;
+  const uint64_t gmax = (bank_head + kCopyThreads * kCopyUnroll - 1) / (kCopyThreads * kCopyUnroll);
+  if (gx > gmax) gx = gmax;
+  if (gx < 1) gx = 1;
+  dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(segs));
+  seg_copy_kernel<<<grid, kCopyThreads, 0, st>>>(p, sel, flag);
+  count_launch();
+  return check_launch("bank/cache copy");
+}
+
+}  // namespace prsink
+
+using namespace prsink;
+
+extern "C" int prsink_kv_append(const prsink_layout* layout, const void* k_new,
+                                const void* v_new, void* k_cache, void* v_cache, int dest_slot,
+                                void* stream) {
+  Geometry g;
+  int rc = geometry(layout, &g);
+  if (rc) return rc;
+  if (!k_new || !v_new || !k_cache || !v_cache) {
+    set_error("prsink_kv_append: null pointer");
+    return PRSINK_ERR_ARG;
+  }
+  if (dest_slot < 0 || dest_slot >= g.n_slots) {
+    set_error("prsink_kv_append: dest_slot %d out of range [0, %d)", dest_slot, g.n_slots);
+    return PRSINK_ERR_ARG;
+  }
+  if ((layout->head_dim * 2) % 16) {
+    set_error("prsink_kv_append: head_dim*2 must be a multiple of 16 bytes");
+    return PRSINK_ERR_UNSUPPORTED;
+  }
+  if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) || !aligned16(v_cache)) {
+    set_error("prsink_kv_append: pointers must be 16-byte aligned");
+    return PRSINK_ERR_ALIGN;
+  }
+  const uint64_t n = g.slot_start[dest_slot + 1] - g.slot_start[dest_slot];
+  const uint32_t C = layout->head_dim * 2 / 16;
+  const uint64_t chunks = n * layout->n_heads * C;
+  if (chunks == 0) return PRSINK_OK;
+  dim3 grid(grid_for(chunks), 2);
+  append_kernel<<<grid, kCopyThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new),
+      static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache),
+      static_cast<uint32_t>(chunks), layout->n_heads, C, static_cast<uint64_t>(g.T),
+      static_cast<uint64_t>(g.slot_start[dest_slot]));
+  count_launch();
+  return check_launch("prsink_kv_append");
+}

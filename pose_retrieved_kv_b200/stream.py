@@ -1,0 +1,98 @@
+"""Host-side bookkeeping of a PR-Sink stream on one GPU.
+
+Per block b, in the order the pages give (LiveAnimate digest, pipeline paragraph, inference
+clause): fingerprint the incoming poses and retrieve the most similar bank entry (excluding
+block b-1) into the dynamic sink; run the denoising passes and the Clean KV Update pass, each
+appending the block's raw K/V into ring slot b mod R and attending over the bounded cache;
+then (first ``write_blocks`` blocks) update the memory bank with the clean K/V.
+
+Decisions stay on the device: the retrieved slot, whether the dynamic sink was refilled and
+the bank action are device scalars read by the copy kernels, and the attention kernel reads
+the dynamic sink's source block to know whether that slot holds data.  Nothing here
+synchronises with the host.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import _lib as L
+
+
+def stream_valid_mask(ring_slots: int, b: int) -> int:
+    """Slots that hold data while block b is generated (the dynamic bit is refined on the
+    device from the dynamic sink's source block): the ref sink; the static sink from block 1
+    on (block 0's clean pass fills it); ring slot s once the block it holds, b-R+1+age(s),
+    is >= 0."""
+    R = ring_slots
+    m = (1 << L.SLOT_REF) | (1 << L.SLOT_DYNAMIC)
+    if b >= 1:
+        m |= 1 << L.SLOT_STATIC
+    oldest = b - R + 1
+    for s in range(R):
+        if oldest + (s - oldest) % R >= 0:
+            m |= 1 << (L.SLOT_RING0 + s)
+    return m
+
+
+class PRSinkStream:
+    """Caches, bank and decisions of one stream for ``n_layers`` attention layers."""
+
+    def __init__(self, cfg: dict, n_layers: int, M: int = 5, write_blocks: int = 20,
+                 device="cuda"):
+        self.cfg = dict(cfg)
+        self.n_layers, self.M, self.write_blocks = int(n_layers), int(M), int(write_blocks)
+        self.R = int(cfg["ring_slots"])
+        lay = L.make_layout(**{**self.cfg, "block_index": 0, "valid_mask": 0})
+        self.L_f, self.L_blk, self.L_ref, self.T = L.prsink_layout_tokens(lay)
+        H, d = int(cfg["n_heads"]), int(cfg["head_dim"])
+        dev = torch.device(device)
+        bf = torch.bfloat16
+        self.cache_kv = torch.zeros((n_layers, 2, H, self.T, d), dtype=bf, device=dev)
+        self.bank_kv = torch.zeros((n_layers, M, 2, H, self.L_blk, d), dtype=bf, device=dev)
+        self.bank_phi = torch.zeros((M, L.FP_DIM), dtype=torch.float32, device=dev)
+        self.bank_src = torch.full((M,), -1, dtype=torch.int64, device=dev)
+        self.bank_count = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.dyn_src = torch.full((1,), -1, dtype=torch.int64, device=dev)
+        self.phi = torch.zeros(L.FP_DIM, dtype=torch.float32, device=dev)
+        self.r = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.score = torch.zeros(1, dtype=torch.float32, device=dev)
+        self.copied = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.action = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.b = 0
+
+    def layout(self, b: int = None) -> L.Layout:
+        b = self.b if b is None else b
+        return L.make_layout(**{**self.cfg, "block_index": b,
+                                "valid_mask": stream_valid_mask(self.R, b)})
+
+    def kv(self, layer: int):
+        return self.cache_kv[layer, 0], self.cache_kv[layer, 1]
+
+    def set_ref(self, layer: int, k_ref, v_ref, stream=None):
+        k, v = self.kv(layer)
+        L.prsink_kv_append(self.layout(), k_ref, v_ref, k, v, L.SLOT_REF, stream)
+
+    def begin_block(self, kp, frame_ok, stream=None):
+        """Fingerprint (kp f32 [3][62][3], frame_ok u8 [3], on the device) and retrieval."""
+        L.prsink_fingerprint(kp, frame_ok, self.phi, stream)
+        L.prsink_retrieve(self.layout(), self.phi, self.bank_phi, self.bank_src,
+                          self.bank_count, self.M, self.b - 1, self.r, self.score, self.copied,
+                          self.dyn_src, self.bank_kv, self.cache_kv, self.n_layers, stream)
+
+    def layer_pass(self, layer: int, q, k_new, v_new, out, lse=None, clean: bool = False,
+                   stream=None):
+        """Append this pass's raw K/V into ring slot b mod R (and, on block 0's clean pass,
+        into the static sink), then attend."""
+        lay = self.layout()
+        k, v = self.kv(layer)
+        L.prsink_kv_append(lay, k_new, v_new, k, v, L.SLOT_RING0 + self.b % self.R, stream)
+        if clean and self.b == 0:
+            L.prsink_kv_append(lay, k_new, v_new, k, v, L.SLOT_STATIC, stream)
+        L.prsink_attention(lay, q, k, v, out, lse, self.dyn_src, stream)
+
+    def end_block(self, stream=None):
+        """Bank update with the clean K/V of block b, then advance to block b+1."""
+        L.prsink_bank_update(self.layout(), self.bank_phi, self.bank_src, self.bank_count,
+                             self.M, self.phi, self.b, self.write_blocks, self.action,
+                             self.cache_kv, self.bank_kv, self.n_layers, stream)
+        self.b += 1

@@ -1,0 +1,98 @@
+"""The C ABI library loads, exports every symbol ``include/prsink.h`` declares, and rejects
+invalid arguments on the host before launching anything (CPU only: no compute call)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import pose_retrieved_kv_b200 as P
+import synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "prsink.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(prsink_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for n in ("prsink_attention", "prsink_kv_append", "prsink_retrieve", "prsink_bank_update",
+              "prsink_fingerprint", "prsink_sync_status"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(P.LIB_PATH)
+    for name in _declared():
+        assert hasattr(lib, name), name
+    out = subprocess.run(["nm", "-D", "--defined-only", P.LIB_PATH], capture_output=True,
+                         text=True).stdout
+    exported = set(re.findall(r"\bT (prsink_\w+)", out))
+    assert set(_declared()) <= exported
+    assert set(P.exported_symbols()) <= exported
+
+
+def test_build_targets_sm100a():
+    from pose_retrieved_kv_b200 import build
+    assert build.ARCH == ["-gencode", "arch=compute_100a,code=sm_100a"]
+
+
+def test_layout_tokens_match_slot_arithmetic():
+    for name, T in [("tiny", 256), ("480x480", 14400), ("384x672", 16128), ("384x672_r4", 19152)]:
+        lay = P.make_layout(**synth.preset(name))
+        L_f, L_blk, L_ref, TT = P.prsink_layout_tokens(lay)
+        assert TT == T and L_blk == 3 * L_f and L_ref == L_f
+
+
+@pytest.mark.parametrize("bad", [dict(n_heads=0), dict(ring_slots=0), dict(ring_slots=9),
+                                 dict(rope_split=(44, 42, 40)), dict(rope_split=(43, 43, 42)),
+                                 dict(rope_mode=2), dict(block_index=-1), dict(rope_base=0.0)])
+def test_invalid_layout_rejected(bad):
+    lay = P.make_layout(**{**synth.preset("480x480"), **bad})
+    with pytest.raises(P.PRSinkError) as e:
+        P.prsink_layout_tokens(lay)
+    assert e.value.code == P.PRSINK_ERR_ARG
+
+
+def _lib():
+    return P._lib._lib
+
+
+def test_null_and_range_errors_do_not_launch():
+    lib = _lib()
+    lay = P.make_layout(**synth.preset("tiny"))
+    before = P.prsink_launch_count()
+    assert lib.prsink_attention(ctypes.byref(lay), None, None, None, None, None, None,
+                                None) == P.PRSINK_ERR_ARG
+    assert lib.prsink_kv_append(ctypes.byref(lay), 16, 16, 16, 16, 99, None) == P.PRSINK_ERR_ARG
+    assert lib.prsink_kv_append(ctypes.byref(lay), 16, 16, 16, 16, -1, None) == P.PRSINK_ERR_ARG
+    assert lib.prsink_kv_append(ctypes.byref(lay), 17, 16, 16, 16, 3, None) == P.PRSINK_ERR_ALIGN
+    assert lib.prsink_attention(ctypes.byref(lay), 16, 16, 16, 24, None, None,
+                                None) == P.PRSINK_ERR_ALIGN
+    lay96 = P.make_layout(**{**synth.preset("tiny"), "head_dim": 96, "rope_split": (96, 0, 0)})
+    assert lib.prsink_attention(ctypes.byref(lay96), 16, 16, 16, 16, None, None,
+                                None) == P.PRSINK_ERR_UNSUPPORTED
+    assert lib.prsink_retrieve(None, 16, 16, 16, 16, 0, 0, 16, 16, 16, 16, None, None, 0,
+                               None) == P.PRSINK_ERR_ARG          # M = 0
+    assert lib.prsink_retrieve(None, 16, 16, 16, 16, 33, 0, 16, 16, 16, 16, None, None, 0,
+                               None) == P.PRSINK_ERR_ARG          # M > 32
+    assert lib.prsink_retrieve(None, 16, 16, 16, 16, 5, 0, 16, 16, 16, 16, 16, None, 1,
+                               None) == P.PRSINK_ERR_ARG          # copy without a layout
+    assert lib.prsink_bank_update(ctypes.byref(lay), 16, 16, 16, 5, 16, -1, 20, 16, None,
+                                  None, 0, None) == P.PRSINK_ERR_ARG   # b < 0
+    assert lib.prsink_fingerprint(None, 16, 16, None) == P.PRSINK_ERR_ARG
+    assert P.prsink_launch_count() == before
+    assert "null" in P.prsink_last_error() or P.prsink_last_error()
+
+
+def test_rope_table_limit_reported():
+    # 1-D RoPE over a large frame needs a table that does not fit in shared memory
+    lay = P.make_layout(**{**synth.preset("480x480"), "rope_mode": 1, "rope_split": (128, 0, 0)})
+    assert _lib().prsink_attention(ctypes.byref(lay), 16, 16, 16, 16, None, None,
+                                   None) == P.PRSINK_ERR_UNSUPPORTED
