@@ -235,6 +235,67 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     return res
 
 
+def run_kernel_only(args, local_rank: int):
+    """Time one kernel alone (``--only attention|append``) at the workload's sizes: W warm-up
+    launches, then K launches on fresh buffers (a rotating set larger than L2)."""
+    import torch
+
+    import pose_retrieved_kv_b200 as P
+    import synth
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    cfg = synth.preset(args.config, block_index=1000, valid_mask=0xFF)
+    lay = P.make_layout(**cfg)
+    _, lblk, _, T = P.prsink_layout_tokens(lay)
+    H, d = cfg["n_heads"], cfg["head_dim"]
+    nbuf = 2
+    q = [synth.normal_bf16((lblk, H, d), 5 + i, 0).to(dev) for i in range(nbuf)]
+    k = [synth.normal_bf16((H, T, d), 5 + i, 1).to(dev) for i in range(nbuf)]
+    v = [synth.normal_bf16((H, T, d), 5 + i, 2).to(dev) for i in range(nbuf)]
+    out = torch.empty((lblk, H, d), dtype=torch.bfloat16, device=dev)
+
+    def launch(i):
+        j = i % nbuf
+        if args.only == "attention":
+            P.prsink_attention(lay, q[j], k[j], v[j], out)
+        else:
+            P.prsink_kv_append(lay, q[j], q[(j + 1) % nbuf], k[j], v[j], P.SLOT_RING0)
+
+    for i in range(args.warmup):
+        launch(i)
+    torch.cuda.synchronize()
+    times = []
+    for i in range(args.steps):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        launch(args.warmup + i)
+        e1.record()
+        times.append((e0, e1))
+    torch.cuda.synchronize()
+    if P.prsink_sync_status() != P.PRSINK_OK:
+        raise RuntimeError("device status reported a timeout")
+    ms = [a.elapsed_time(b) for a, b in times]
+    peaks = _peaks()
+    avg = statistics.mean(ms)
+    if args.only == "attention":
+        work = 4.0 * lblk * T * d * H
+        ach = work / (avg / 1e3) / 1e12
+        roof = {"bound": "tensor", "achieved": round(ach, 1), "peak": peaks["bf16"],
+                "unit": "TFLOP/s", "frac": round(ach / peaks["bf16"], 4),
+                "peak_source": f"{peaks['source']} bf16_tflops (burst)"}
+    else:
+        work = 2.0 * 2 * lblk * H * d * 2                   # K and V: read + write
+        ach = work / (avg / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm"],
+                "unit": "GB/s", "frac": round(ach / peaks["hbm"], 4),
+                "peak_source": f"{peaks['source']} hbm_gbs"}
+    return {"kernel": args.only, "config": args.config, "avg_ms": round(avg, 4),
+            "min_ms": round(min(ms), 4), "max_ms": round(max(ms), 4), "launches": len(ms),
+            "roofline": roof}
+
+
 def run_e2e(args, st, qkv, kp_all, ok_all, dev, world):
     """Same step through the public API with pinned HOST inputs and outputs: every step copies
     its poses and per-pass Q/K/V from the host and reads every attention output back.  Copies
@@ -415,6 +476,8 @@ def main():
     ap.add_argument("--cpu-heads", type=int, default=4)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", choices=["attention", "append"], default=None,
+                    help="time one kernel alone at the workload's sizes (for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -423,7 +486,9 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if world != args.gpus:
         world = max(world, 1)
-    if args.impl == "reference":
+    if args.only:
+        res = run_kernel_only(args, local_rank)
+    elif args.impl == "reference":
         res = run_reference(args, rank, world)
     else:
         import torch.distributed as dist

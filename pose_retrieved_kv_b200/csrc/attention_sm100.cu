@@ -1,17 +1,21 @@
 // PR-Sink attention for sm_100a: TMA-staged K/V tiles from the slot-indexed cache, RoPE of the
 // raw keys fused between the TMA landing and the tensor-core read ("RoPE follow"), tcgen05 MMAs
-// with accumulators in tensor memory, fp32 online softmax, no materialised score matrix.
+// with S, P and O in tensor memory, fp32 online softmax, no materialised score matrix.
 //
-// One CTA computes one 128-query tile of one head.  Warp roles (320 threads):
-//   warps 0-3  softmax: thread t owns query row t (= TMEM lane t); reads S from TMEM, keeps
-//              the running max / sum, writes P (bf16) to shared memory, rescales O in TMEM
-//              when the max grows by more than 2^8, and finally normalises and stores O;
-//   warp  4    TMA producer: Q once, then K and V tiles into a 2-stage ring;
-//   warp  5    MMA issuer: S = Q K^T into one of two TMEM score buffers, O += P V;
-//   warps 6-9  rotation: rotate Q once and every K tile in place at the keys' current
-//              logical positions (interleaved RoFormer pairs, per-axis tables in shared
-//              memory), zero the rows of empty slots, and hand the tile to the MMA warp.
-// Key tiles run over the physical rows of the cache; softmax attention does not depend on the
+// One CTA computes 256 queries (two 128-row tiles Q0, Q1) of one head, ping-ponging the two
+// tiles so that the tensor core works on one tile while the other tile's softmax runs.
+// Warp roles (512 threads; setmaxnreg gives the softmax warps 192 registers, the rotation
+// warps 56 and the producer / MMA warps 72):
+//   warps 0-3   softmax of Q0, warps 4-7 softmax of Q1: thread t owns query row t (TMEM lane
+//               t); it reads S from TMEM, keeps the running max and sum, writes P as bf16 back
+//               into the S columns (the A operand of the P.V MMA), rescales O in TMEM when the
+//               max grew by more than 2^8, and finally normalises and stores O;
+//   warps 8-11  rotation: rotate Q0/Q1 once and every K tile in place at the keys' current
+//               logical positions (interleaved RoFormer pairs, per-axis cos/sin tables in
+//               shared memory); zero the K and V rows of empty slots in boundary tiles;
+//   warp  12    TMA producer: Q once, then K and V tiles, each through its own 2-stage ring;
+//   warp  13    MMA issuer: per key tile j, P0(j-1).V, S0(j) = Q0 K^T, P1(j-1).V, S1(j).
+// Key tiles run over the physical rows of the cache: softmax attention does not depend on the
 // order of the keys, only on their positions, so each key is rotated at the position of its
 // logical slot and no gather is needed.  Tiles inside empty slots are skipped.
 #include <cuda.h>
@@ -25,12 +29,13 @@
 namespace prsink {
 namespace attn {
 
-constexpr int BM = 128;                 // queries per CTA
+constexpr int BM = 128;                 // rows of one query tile (= TMEM lanes)
+constexpr int NQ = 2;                   // query tiles per CTA
 constexpr int BN = 128;                 // keys per tile
-constexpr int kThreads = 320;
-constexpr int kProducerWarp = 4;
-constexpr int kMmaWarp = 5;
-constexpr int kRotWarp0 = 6;
+constexpr int kThreads = 512;
+constexpr int kRotWarp0 = 8;
+constexpr int kProducerWarp = 12;
+constexpr int kMmaWarp = 13;
 constexpr int kMaxSlots = 3 + PRSINK_MAX_RING;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kTableMaxBytes = 32 * 1024;
@@ -57,28 +62,36 @@ struct Params {
 };
 
 enum Bar {
-  B_QFULL = 0, B_QREADY = 1, B_KVFULL = 2, B_KREADY = 4, B_KVEMPTY = 6, B_SFULL = 8,
-  B_SFREE = 10, B_PFULL = 12, B_ODONE = 13, B_FINAL = 14, B_COUNT = 15
+  B_QFULL = 0, B_QREADY = 1,
+  B_KFULL = 2, B_KREADY = 4, B_KEMPTY = 6,
+  B_VFULL = 8, B_VFIX = 10, B_VEMPTY = 12,
+  B_SFULL = 14, B_PFULL = 16, B_ODONE = 18,
+  B_FINAL = 20, B_COUNT = 21
 };
 
 template <int D>
 struct Layout {
-  static constexpr int kPanels = D / 64;
   static constexpr int kPanelBytes = 128 * 128;          // 128 rows x 128 B (64 bf16)
-  static constexpr int kTileBytes = kPanels * kPanelBytes;
-  static constexpr int kQ = 0;
-  static constexpr int kK = kQ + kTileBytes;             // 2 stages
+  static constexpr int kTileBytes = (D / 64) * kPanelBytes;
+  static constexpr int kQ = 0;                           // NQ query tiles
+  static constexpr int kK = kQ + NQ * kTileBytes;        // 2 stages
   static constexpr int kV = kK + 2 * kTileBytes;         // 2 stages
-  static constexpr int kP = kV + 2 * kTileBytes;         // 128 x 128 bf16, 2 panels
-  static constexpr int kTab = kP + 2 * kPanelBytes;
+  static constexpr int kTab = kV + 2 * kTileBytes;
   static constexpr uint32_t kIdescS = idesc_bf16_f32(128, BN, false, false);
   static constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, false, true);
+  __host__ __device__ static constexpr uint32_t col_s(int qt) { return qt * 128; }        // S, then P (bf16 pairs)
+  __host__ __device__ static constexpr uint32_t col_o(int qt) { return 256 + qt * D; }
 };
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&b);
 }
 
 __device__ __forceinline__ bool tile_live(int n, unsigned vm, const Params& p) {
@@ -114,7 +127,7 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64
 template <int D>
 __device__ __forceinline__ void rotate_row(uint8_t* tile, int r, int frame, int tok, bool zero,
                                            const float2* __restrict__ tab, const Params& p) {
-  const int y = tok / p.grid_w, x = tok - (tok / p.grid_w) * p.grid_w;
+  const int y = tok / p.grid_w, x = tok - y * p.grid_w;
   const float2* rowT;
   const float2* rowH;
   const float2* rowW;
@@ -130,7 +143,7 @@ __device__ __forceinline__ void rotate_row(uint8_t* tile, int r, int frame, int 
   const int r0 = p.rd[0], r01 = p.rd[0] + p.rd[1];
 #pragma unroll
   for (int pp = 0; pp < D / 64; ++pp) {
-#pragma unroll
+#pragma unroll 2
     for (int c = 0; c < 8; ++c) {
       uint4* ptr = reinterpret_cast<uint4*>(tile + pp * 16384 + r * 128 + ((c ^ (r & 7)) << 4));
       if (zero) {
@@ -149,12 +162,9 @@ __device__ __forceinline__ void rotate_row(uint8_t* tile, int r, int frame, int 
           const float2 a = rowT[P], b = rowH[P];
           cs = make_float2(a.x * b.x - a.y * b.y, a.y * b.x + a.x * b.y);
         }
-        __nv_bfloat162 pr = *reinterpret_cast<__nv_bfloat162*>(&w[i]);
-        const float x0 = __low2float(pr), x1 = __high2float(pr);
-        const float y0 = x0 * cs.x - x1 * cs.y;
-        const float y1 = x0 * cs.y + x1 * cs.x;
-        pr = __floats2bfloat162_rn(y0, y1);
-        w[i] = *reinterpret_cast<uint32_t*>(&pr);
+        const float x0 = __uint_as_float(w[i] << 16);
+        const float x1 = __uint_as_float(w[i] & 0xFFFF0000u);
+        w[i] = pack_bf16(x0 * cs.x - x1 * cs.y, x0 * cs.y + x1 * cs.x);
       }
       *ptr = v;
     }
@@ -177,25 +187,27 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
   const uint32_t raw = smem_u32(dsmem);
   const uint32_t sb = (raw + 1023u) & ~1023u;            // 1 KB aligned base (swizzle atoms)
   uint8_t* gb = dsmem + (sb - raw);
-  const uint32_t sQ = sb + LY::kQ, sK = sb + LY::kK, sV = sb + LY::kV, sP = sb + LY::kP;
+  const uint32_t sQ = sb + LY::kQ, sK = sb + LY::kK, sV = sb + LY::kV;
   float2* tab = reinterpret_cast<float2*>(gb + LY::kTab);
   auto bar = [&](int i) { return smem_u32(&bars[i]); };
 
-  const int q0 = blockIdx.x * BM;
+  const int q0 = blockIdx.x * (NQ * BM);
   const int h = blockIdx.y;
 
   if (threadIdx.x == 0) {
     mbar_init(bar(B_QFULL), 1);
     mbar_init(bar(B_QREADY), 128);
     for (int s = 0; s < 2; ++s) {
-      mbar_init(bar(B_KVFULL + s), 1);
+      mbar_init(bar(B_KFULL + s), 1);
       mbar_init(bar(B_KREADY + s), 128);
-      mbar_init(bar(B_KVEMPTY + s), 1);
+      mbar_init(bar(B_KEMPTY + s), 1);
+      mbar_init(bar(B_VFULL + s), 1);
+      mbar_init(bar(B_VFIX + s), 128);
+      mbar_init(bar(B_VEMPTY + s), 1);
       mbar_init(bar(B_SFULL + s), 1);
-      mbar_init(bar(B_SFREE + s), 128);
+      mbar_init(bar(B_PFULL + s), 128);
+      mbar_init(bar(B_ODONE + s), 1);
     }
-    mbar_init(bar(B_PFULL), 128);
-    mbar_init(bar(B_ODONE), 1);
     mbar_init(bar(B_FINAL), 1);
     ab.flag = 0;
     unsigned vm = p.valid_mask;
@@ -224,9 +236,11 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
       if (e < p.tab_h_off) { pos = (e / (D / 2)) * p.L_f; j = e % (D / 2); }
       else { const int f = e - p.tab_h_off; pos = f / (D / 2); j = f % (D / 2); }
     }
-    const double theta = exp2(-(2.0 * j / da) * p.log2_base);
+    // angle / pi, so that the reduction of the argument is exact (sincospi)
+    const double turns = static_cast<double>(pos) * exp2(-(2.0 * j / da) * p.log2_base) *
+                         0.31830988618379067154;
     double sn, cs;
-    sincos(static_cast<double>(pos) * theta, &sn, &cs);
+    sincospi(turns, &sn, &cs);
     tab[e] = make_float2(static_cast<float>(cs), static_cast<float>(sn));
   }
   tc_fence_before();
@@ -238,75 +252,108 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
   const uint64_t deadline = globaltimer() + p.timeout_ns;
   const int n_tiles = (p.T + BN - 1) / BN;
 
-  if (warp == kProducerWarp) {
-    // ------------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      mbar_arrive_expect_tx(bar(B_QFULL), LY::kTileBytes);
-      for (int pp = 0; pp < D / 64; ++pp)
-        tma_load_3d(sQ + pp * 16384, &tm_q, bar(B_QFULL), pp * 64, h, q0);
-      int it = 0;
-      int issued[2] = {-1, -1};
+  if (warp >= kProducerWarp) {
+    setmaxnreg_dec<72>();
+    if (warp == kProducerWarp && lane == 0) {
+      // ---------------------------------------------------------------- TMA producer
+      mbar_arrive_expect_tx(bar(B_QFULL), NQ * LY::kTileBytes);
+      for (int qt = 0; qt < NQ; ++qt)
+        for (int pp = 0; pp < D / 64; ++pp)
+          tma_load_3d(sQ + qt * LY::kTileBytes + pp * 16384, &tm_q, bar(B_QFULL), pp * 64, h,
+                      q0 + qt * BM);
+      int j = 0;
       for (int n = 0; n < n_tiles; ++n) {
         if (!tile_live(n, vm, p)) continue;
-        const int st = it & 1;
-        if (it >= 2 && !mbar_wait(bar(B_KVEMPTY + st), ((it >> 1) - 1) & 1, &ab, deadline, p.status))
-          break;
-        mbar_arrive_expect_tx(bar(B_KVFULL + st), 2 * LY::kTileBytes);
-        for (int pp = 0; pp < D / 64; ++pp) {
-          tma_load_3d(sK + st * LY::kTileBytes + pp * 16384, &tm_k, bar(B_KVFULL + st), pp * 64,
+        const int st = j & 1;
+        const uint32_t par = ((j >> 1) - 1) & 1;
+        if (j >= 2 && !mbar_wait(bar(B_KEMPTY + st), par, &ab, deadline, p.status)) break;
+        mbar_arrive_expect_tx(bar(B_KFULL + st), LY::kTileBytes);
+        for (int pp = 0; pp < D / 64; ++pp)
+          tma_load_3d(sK + st * LY::kTileBytes + pp * 16384, &tm_k, bar(B_KFULL + st), pp * 64,
                       n * BN, h);
-          tma_load_3d(sV + st * LY::kTileBytes + pp * 16384, &tm_v, bar(B_KVFULL + st), pp * 64,
+        if (j >= 2 && !mbar_wait(bar(B_VEMPTY + st), par, &ab, deadline, p.status)) break;
+        mbar_arrive_expect_tx(bar(B_VFULL + st), LY::kTileBytes);
+        for (int pp = 0; pp < D / 64; ++pp)
+          tma_load_3d(sV + st * LY::kTileBytes + pp * 16384, &tm_v, bar(B_VFULL + st), pp * 64,
                       n * BN, h);
-        }
-        issued[st] = it;
-        ++it;
+        ++j;
       }
       if (ab.flag) {     // let copies in flight land before the CTA's shared memory goes away
+        // the last loads issued into stage s belong to iteration j-1-((j-1-s)&1)
         drain_wait(bar(B_QFULL), 0, 100000000ull);
-        for (int s = 0; s < 2; ++s)
-          if (issued[s] >= 0) drain_wait(bar(B_KVFULL + s), (issued[s] >> 1) & 1, 100000000ull);
+        for (int s = 0; s < 2; ++s) {
+          const int last = j - 1 - ((j - 1 - s) & 1);
+          if (last >= 0) {
+            drain_wait(bar(B_KFULL + s), (last >> 1) & 1, 100000000ull);
+            drain_wait(bar(B_VFULL + s), (last >> 1) & 1, 100000000ull);
+          }
+        }
       }
-    }
-  } else if (warp == kMmaWarp) {
-    // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    } else if (warp == kMmaWarp && lane == 0) {
+      // ---------------------------------------------------------------- MMA issuer
       bool ok = mbar_wait(bar(B_QREADY), 0, &ab, deadline, p.status);
       tc_fence_after();
-      const uint32_t tO = tmem + 256;
-      auto issue_pv = [&](int j) -> bool {
-        if (!mbar_wait(bar(B_PFULL), j & 1, &ab, deadline, p.status)) return false;
-        tc_fence_after();
-        const uint32_t v_base = sV + (j & 1) * LY::kTileBytes;
-#pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint64_t a = sdesc_sw128(sP + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-          const uint64_t b = sdesc_sw128(v_base + kk * 2048, 16384, 1024);
-          umma_ss(tO, a, b, LY::kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
-        }
-        umma_commit(bar(B_ODONE));
-        umma_commit(bar(B_KVEMPTY + (j & 1)));
-        return true;
-      };
-      int it = 0;
-      for (int n = 0; ok && n < n_tiles; ++n) {
-        if (!tile_live(n, vm, p)) continue;
-        const int st = it & 1;
-        if (!mbar_wait(bar(B_KREADY + st), (it >> 1) & 1, &ab, deadline, p.status)) { ok = false; break; }
-        if (it >= 2 && !mbar_wait(bar(B_SFREE + st), ((it >> 1) - 1) & 1, &ab, deadline, p.status)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t tS = tmem + st * 128;
+      int fix0 = 0, fix1 = 0;                              // boundary tiles seen per stage
+      auto s_mma = [&](int qt, int st) {
+        const uint32_t q_base = sQ + qt * LY::kTileBytes;
         const uint32_t k_base = sK + st * LY::kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t a = sdesc_sw128(sQ + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-          const uint64_t b = sdesc_sw128(k_base + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-          umma_ss(tS, a, b, LY::kIdescS, kk > 0 ? 1u : 0u);
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          umma_ss(tmem + LY::col_s(qt), sdesc_sw128(q_base + off, 16, 1024),
+                  sdesc_sw128(k_base + off, 16, 1024), LY::kIdescS, kk > 0 ? 1u : 0u);
         }
-        umma_commit(bar(B_SFULL + st));
-        if (it >= 1 && !issue_pv(it - 1)) { ok = false; break; }
-        ++it;
+      };
+      // O_qt (+)= P_qt(i) V(i); V(i) must have landed (and been fixed up in boundary tiles)
+      auto pv_mma = [&](int qt, int i, bool partial) -> bool {
+        const int st = i & 1;
+        if (qt == 0) {
+          if (!mbar_wait(bar(B_VFULL + st), (i >> 1) & 1, &ab, deadline, p.status)) return false;
+          if (partial) {
+            int& fx = st ? fix1 : fix0;
+            if (!mbar_wait(bar(B_VFIX + st), fx & 1, &ab, deadline, p.status)) return false;
+            ++fx;
+          }
+        }
+        if (!mbar_wait(bar(B_PFULL + qt), i & 1, &ab, deadline, p.status)) return false;
+        tc_fence_after();
+        const uint32_t v_base = sV + st * LY::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk)
+          umma_ts(tmem + LY::col_o(qt), tmem + LY::col_s(qt) + kk * 8,
+                  sdesc_sw128(v_base + kk * 2048, 16384, 1024), LY::kIdescPV,
+                  (i > 0 || kk > 0) ? 1u : 0u);
+        return true;
+      };
+      int j = 0;
+      bool prev_partial = false;
+      for (int n = 0; ok && n < n_tiles; ++n) {
+        if (!tile_live(n, vm, p)) continue;
+        const int st = j & 1;
+        if (!mbar_wait(bar(B_KREADY + st), (j >> 1) & 1, &ab, deadline, p.status)) { ok = false; break; }
+        tc_fence_after();
+        if (j >= 1 && !pv_mma(0, j - 1, prev_partial)) { ok = false; break; }
+        s_mma(0, st);
+        umma_commit(bar(B_SFULL + 0));
+        if (j >= 1) {
+          if (!pv_mma(1, j - 1, prev_partial)) { ok = false; break; }
+          umma_commit(bar(B_VEMPTY + ((j - 1) & 1)));
+        }
+        s_mma(1, st);
+        umma_commit(bar(B_SFULL + 1));
+        umma_commit(bar(B_KEMPTY + st));
+        prev_partial = !tile_full(n, vm, p);
+        ++j;
       }
-      if (ok && it >= 1) issue_pv(it - 1);
+      if (ok && j >= 1) {
+        if (pv_mma(0, j - 1, prev_partial)) {
+          umma_commit(bar(B_ODONE + 0));
+          if (pv_mma(1, j - 1, prev_partial)) {
+            umma_commit(bar(B_VEMPTY + ((j - 1) & 1)));
+            umma_commit(bar(B_ODONE + 1));
+          }
+        }
+      }
       if (ab.flag) {     // wait for every MMA issued so far before TMEM is released
         umma_commit(bar(B_FINAL));
         drain_wait(bar(B_FINAL), 0, 100000000ull);
@@ -314,59 +361,67 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
     }
   } else if (warp >= kRotWarp0) {
     // ------------------------------------------------------------------ rotation
+    setmaxnreg_dec<56>();
     const int rt = threadIdx.x - kRotWarp0 * 32;          // row of the tile, 0..127
     if (mbar_wait(bar(B_QFULL), 0, &ab, deadline, p.status)) {
-      const int qi = q0 + rt;
-      if (qi < p.L_blk)
-        rotate_row<D>(gb + LY::kQ, rt, p.q_frame + qi / p.L_f, qi % p.L_f, false, tab, p);
+      for (int qt = 0; qt < NQ; ++qt) {
+        const int qi = q0 + qt * BM + rt;
+        if (qi < p.L_blk)
+          rotate_row<D>(gb + LY::kQ + qt * LY::kTileBytes, rt, p.q_frame + qi / p.L_f,
+                        qi % p.L_f, false, tab, p);
+      }
       fence_proxy_async_smem();
       mbar_arrive(bar(B_QREADY));
-      int it = 0;
+      int j = 0;
       for (int n = 0; n < n_tiles; ++n) {
         if (!tile_live(n, vm, p)) continue;
-        const int st = it & 1;
-        if (!mbar_wait(bar(B_KVFULL + st), (it >> 1) & 1, &ab, deadline, p.status)) break;
+        const int st = j & 1;
+        if (!mbar_wait(bar(B_KFULL + st), (j >> 1) & 1, &ab, deadline, p.status)) break;
         const int row = n * BN + rt;
+        bool empty = false;
         if (row < p.T) {
           const int s = slot_of(row, p);
           const int u = row - p.slot_start[s];
-          const bool empty = !((vm >> s) & 1u);
-          uint8_t* kt = gb + LY::kK + st * LY::kTileBytes;
-          rotate_row<D>(kt, rt, p.slot_frame[s] + u / p.L_f, u % p.L_f, empty, tab, p);
-          if (empty) rotate_row<D>(gb + LY::kV + st * LY::kTileBytes, rt, 0, 0, true, tab, p);
+          empty = !((vm >> s) & 1u);
+          rotate_row<D>(gb + LY::kK + st * LY::kTileBytes, rt, p.slot_frame[s] + u / p.L_f,
+                        u % p.L_f, empty, tab, p);
         }
         fence_proxy_async_smem();
         mbar_arrive(bar(B_KREADY + st));
-        ++it;
+        if (!tile_full(n, vm, p)) {
+          // boundary tile: empty-slot rows of V may hold anything; P is 0 there, but 0 * NaN
+          // is not, so zero them before the P.V MMA reads the tile
+          if (!mbar_wait(bar(B_VFULL + st), (j >> 1) & 1, &ab, deadline, p.status)) break;
+          if (empty) rotate_row<D>(gb + LY::kV + st * LY::kTileBytes, rt, 0, 0, true, tab, p);
+          fence_proxy_async_smem();
+          mbar_arrive(bar(B_VFIX + st));
+        }
+        ++j;
       }
     }
   } else {
-    // ------------------------------------------------------------------ softmax (warps 0-3)
-    const int t = threadIdx.x;                            // query row = TMEM lane
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-    const uint32_t tO = tmem + lane_off + 256;
+    // ------------------------------------------------------------------ softmax (warps 0-7)
+    setmaxnreg_inc<192>();
+    const int qt = warp >> 2;                             // query tile of this warpgroup
+    const int t = threadIdx.x & (BM - 1);                 // query row = TMEM lane
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_off + LY::col_s(qt);
+    const uint32_t tO = tmem + lane_off + LY::col_o(qt);
+    const float2 scale2 = make_float2(p.scale_log2, p.scale_log2);
     float m = -INFINITY, l = 0.f;
-    int it = 0;
+    int j = 0;
     bool ok = true;
-    uint8_t* prow = gb + LY::kP;
     for (int n = 0; n < n_tiles; ++n) {
       if (!tile_live(n, vm, p)) continue;
-      const int st = it & 1;
-      ok = mbar_wait(bar(B_SFULL + st), (it >> 1) & 1, &ab, deadline, p.status);
+      ok = mbar_wait(bar(B_SFULL + qt), j & 1, &ab, deadline, p.status);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }   // tcgen05.ld is warp-collective
       tc_fence_after();
       uint32_t s[128];
-      const uint32_t tS = tmem + lane_off + st * 128;
       tmem_ld32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
       tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
       tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
       tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
       tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(bar(B_SFREE + st));
-      float x[128];
-#pragma unroll
-      for (int c = 0; c < 128; ++c) x[c] = __uint_as_float(s[c]) * p.scale_log2;
       if (!tile_full(n, vm, p)) {
         // columns of empty slots and past the end of the cache: 4 mask words, built per slot
         const int lo = n * BN;
@@ -392,37 +447,45 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
         }
 #pragma unroll
         for (int c = 0; c < 128; ++c)
-          if (!((mw[c >> 5] >> (c & 31)) & 1u)) x[c] = -INFINITY;
+          if (!((mw[c >> 5] >> (c & 31)) & 1u)) s[c] = __float_as_uint(-INFINITY);
       }
-      float mt = x[0];
+      // row max of the raw scores (scaling by a positive constant keeps the argmax)
+      float mt = fmax3(__uint_as_float(s[0]), __uint_as_float(s[1]), __uint_as_float(s[2]));
 #pragma unroll
-      for (int c = 1; c < 128; ++c) mt = fmaxf(mt, x[c]);
+      for (int c = 3; c < 127; c += 2)
+        mt = fmax3(mt, __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
+      mt = fmaxf(mt, __uint_as_float(s[127])) * p.scale_log2;
       float alpha = 1.f;
       bool rescale = false;
-      if (it == 0) {
+      if (j == 0) {
         m = mt;
       } else if (mt > m + kRescaleThreshold) {
         alpha = ex2(m - mt);
         m = mt;
         rescale = true;
       }
-      float sum = 0.f;
-      uint32_t pk[64];                          // P as bf16 pairs: keeps the rescale in registers
+      // P = 2^(s*scale - m) as bf16 pairs into the S columns (A operand of the P.V MMA):
+      // 32 scores -> 16 packed words -> one 16-column TMEM store
+      const float2 negm = make_float2(-m, -m);
+      float2 sum2 = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int c = 0; c < 128; c += 2) {
-        const float p0 = ex2(x[c] - m), p1 = ex2(x[c + 1] - m);
-        sum += p0 + p1;
-        __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
-        pk[c >> 1] = *reinterpret_cast<uint32_t*>(&b2);
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int c = ch * 32 + 2 * i;
+          const float2 e2 = ffma2(make_float2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])),
+                                  scale2, negm);
+          const float2 pr = make_float2(ex2(e2.x), ex2(e2.y));
+          sum2 = fadd2(sum2, pr);
+          pk[i] = pack_bf16(pr.x, pr.y);
+        }
+        tmem_st16(tS + ch * 16, pk);
       }
-      l = l * alpha + sum;
-      if (it >= 1) {
-        ok = mbar_wait(bar(B_ODONE), (it - 1) & 1, &ab, deadline, p.status);
-        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-        tc_fence_after();
-      }
+      l = l * alpha + (sum2.x + sum2.y);
       if (__any_sync(0xffffffffu, rescale)) {   // rows that keep their max scale by alpha = 1
-#pragma unroll
+        // O_qt holds every P.V up to tile j-1: the S(j) commit completed after them
+#pragma unroll 1
         for (int cc = 0; cc < D / 32; ++cc) {
           uint32_t o[32];
           tmem_ld32(tO + cc * 32, o);
@@ -431,34 +494,24 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
           for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
           tmem_st32(tO + cc * 32, o);
         }
-        tmem_wait_st();
       }
-#pragma unroll
-      for (int pp = 0; pp < 2; ++pp) {
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const int k = pp * 32 + c * 4;
-          *reinterpret_cast<uint4*>(prow + pp * 16384 + t * 128 + ((c ^ (t & 7)) << 4)) =
-              make_uint4(pk[k], pk[k + 1], pk[k + 2], pk[k + 3]);
-        }
-      }
-      fence_proxy_async_smem();
+      tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar(B_PFULL));
-      ++it;
+      mbar_arrive(bar(B_PFULL + qt));
+      ++j;
     }
     // epilogue: O / l -> bf16, one 2*D-byte row per thread
-    const int qi = q0 + t;
+    const int qi = q0 + qt * BM + t;
     float inv = 0.f;
     bool have = false;
-    if (__all_sync(0xffffffffu, ok) && it > 0) {
-      have = mbar_wait(bar(B_ODONE), (it - 1) & 1, &ab, deadline, p.status);
+    if (__all_sync(0xffffffffu, ok) && j > 0) {
+      have = mbar_wait(bar(B_ODONE + qt), 0, &ab, deadline, p.status);
       have = __all_sync(0xffffffffu, have);
       tc_fence_after();
       inv = l > 0.f ? 1.f / l : 0.f;
     }
     __nv_bfloat16* orow = p.out + (static_cast<size_t>(qi) * p.H + h) * D;
-#pragma unroll
+#pragma unroll 1
     for (int cc = 0; cc < D / 32; ++cc) {
       uint32_t o[32];
       if (have) {                     // warp-uniform
@@ -471,15 +524,11 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
       if (qi < p.L_blk) {
 #pragma unroll
         for (int i = 0; i < 32; i += 8) {
-          __nv_bfloat162 b0 = __floats2bfloat162_rn(__uint_as_float(o[i + 0]) * inv, __uint_as_float(o[i + 1]) * inv);
-          __nv_bfloat162 b1 = __floats2bfloat162_rn(__uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
-          __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(o[i + 4]) * inv, __uint_as_float(o[i + 5]) * inv);
-          __nv_bfloat162 b3 = __floats2bfloat162_rn(__uint_as_float(o[i + 6]) * inv, __uint_as_float(o[i + 7]) * inv);
           uint4 v;
-          v.x = *reinterpret_cast<uint32_t*>(&b0);
-          v.y = *reinterpret_cast<uint32_t*>(&b1);
-          v.z = *reinterpret_cast<uint32_t*>(&b2);
-          v.w = *reinterpret_cast<uint32_t*>(&b3);
+          v.x = pack_bf16(__uint_as_float(o[i + 0]) * inv, __uint_as_float(o[i + 1]) * inv);
+          v.y = pack_bf16(__uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
+          v.z = pack_bf16(__uint_as_float(o[i + 4]) * inv, __uint_as_float(o[i + 5]) * inv);
+          v.w = pack_bf16(__uint_as_float(o[i + 6]) * inv, __uint_as_float(o[i + 7]) * inv);
           *reinterpret_cast<uint4*>(orow + cc * 32 + i) = v;
         }
       }
@@ -560,7 +609,7 @@ static int launch(const prsink_layout* L, const Geometry& g, const void* q, cons
       return check_launch("prsink_attention: shared memory attribute");
     attr_bytes[dev] = smem;
   }
-  dim3 grid((g.L_blk + BM - 1) / BM, L->n_heads);
+  dim3 grid((g.L_blk + NQ * BM - 1) / (NQ * BM), L->n_heads);
   prsink_attention_kernel<D><<<grid, kThreads, smem, st>>>(mq, mk, mv, p);
   count_launch();
   return check_launch("prsink_attention");
