@@ -38,7 +38,8 @@ constexpr int kProducerWarp = 12;
 constexpr int kMmaWarp = 13;
 constexpr int kMaxSlots = 3 + PRSINK_MAX_RING;
 constexpr uint32_t kTmemCols = 512;
-constexpr int kTableMaxBytes = 32 * 1024;
+constexpr int kTableMaxBytes = 28 * 1024;
+constexpr int kMaxTiles = 1024;             // key tiles per call (T <= 131072)
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale O when the max grows > 2^8
 
 struct Params {
@@ -52,6 +53,7 @@ struct Params {
   int rd[3];                            // rotated pairs per axis (1-D: D/2, 0, 0)
   int n_frames;                         // frames of the logical layout
   int tab_h_off, tab_w_off, tab_entries;  // float2 offsets of the tables
+  int step_y, step_x;                   // a step of BN tokens within a frame: rows, columns
   double log2_base;
   float scale_log2;                     // log2(e) / sqrt(d)
   __nv_bfloat16* out;
@@ -123,11 +125,14 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64
 }
 
 // Rotate one 128-byte-swizzled row (D bf16 over D/64 panels) in place at position
-// (frame, tok); or zero it when `zero` is set.
-template <int D>
-__device__ __forceinline__ void rotate_row(uint8_t* tile, int r, int frame, int tok, bool zero,
-                                           const float2* __restrict__ tab, const Params& p) {
-  const int y = tok / p.grid_w, x = tok - y * p.grid_w;
+// (frame, tok); or zero it when `zero` is set.  RT, RH: pairs of the t and h axes when known
+// at compile time (3-D RoPE), 0 to read the split from the parameters.
+template <int D, int RT, int RH>
+__device__ __forceinline__ void rotate_row(uint8_t* tile, int r, int frame, int y, int x,
+                                           bool zero, const float2* __restrict__ tab,
+                                           const Params& p) {
+  // tables are [position][pair]: a row pointer per axis plus a compile-time pair offset; the
+  // w-axis rows are 21 float2 apart, so a half-warp of consecutive columns hits distinct banks
   const float2* rowT;
   const float2* rowH;
   const float2* rowW;
@@ -137,13 +142,14 @@ __device__ __forceinline__ void rotate_row(uint8_t* tile, int r, int frame, int 
     rowW = tab + p.tab_w_off + x * p.rd[2];
   } else {
     rowT = tab + frame * (D / 2);                  // angle of frame*L_f
-    rowH = tab + p.tab_h_off + tok * (D / 2);      // angle of the in-frame token index
+    rowH = tab + p.tab_h_off + (y * p.grid_w + x) * (D / 2);   // in-frame token angle
     rowW = nullptr;
   }
-  const int r0 = p.rd[0], r01 = p.rd[0] + p.rd[1];
+  const int r0 = RT > 0 ? RT : p.rd[0];
+  const int r01 = RT > 0 ? RT + RH : p.rd[0] + p.rd[1];
 #pragma unroll
   for (int pp = 0; pp < D / 64; ++pp) {
-#pragma unroll 2
+#pragma unroll
     for (int c = 0; c < 8; ++c) {
       uint4* ptr = reinterpret_cast<uint4*>(tile + pp * 16384 + r * 128 + ((c ^ (r & 7)) << 4));
       if (zero) {
@@ -156,7 +162,9 @@ __device__ __forceinline__ void rotate_row(uint8_t* tile, int r, int frame, int 
       for (int i = 0; i < 4; ++i) {
         const int P = pp * 32 + c * 4 + i;
         float2 cs;
-        if (p.rope_mode == 3) {
+        if (RT > 0) {                     // axis of pair P fixed at compile time
+          cs = P < RT ? rowT[P] : (P < RT + RH ? rowH[P - RT] : rowW[P - RT - RH]);
+        } else if (p.rope_mode == 3) {
           cs = P < r0 ? rowT[P] : (P < r01 ? rowH[P - r0] : rowW[P - r01]);
         } else {
           const float2 a = rowT[P], b = rowH[P];
@@ -171,7 +179,7 @@ __device__ __forceinline__ void rotate_row(uint8_t* tile, int r, int frame, int 
   }
 }
 
-template <int D>
+template <int D, int RT, int RH>
 __global__ void __launch_bounds__(kThreads, 1)
 prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
                         const __grid_constant__ CUtensorMap tm_k,
@@ -182,6 +190,9 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
   __shared__ uint32_t tmem_base_s;
   __shared__ AbortState ab;
   __shared__ unsigned vmask_s;
+  __shared__ uint8_t tile_flag[kMaxTiles];       // bit 0: holds a valid key, bit 1: boundary
+  __shared__ uint16_t tile_list[kMaxTiles];      // live tiles in order; bit 15: boundary tile
+  __shared__ int n_live_s;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t raw = smem_u32(dsmem);
@@ -215,6 +226,10 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
     vmask_s = vm;
     fence_barrier_init();
   }
+  __syncthreads();
+  const int n_tiles = (p.T + BN - 1) / BN;
+  for (int n = threadIdx.x; n < n_tiles; n += kThreads)
+    tile_flag[n] = (tile_live(n, vmask_s, p) ? 1 : 0) | (tile_full(n, vmask_s, p) ? 0 : 2);
   if (warp == kProducerWarp && lane == 0) {
     prefetch_tmap(&tm_q);
     prefetch_tmap(&tm_k);
@@ -225,6 +240,8 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
     tmem_relinquish();
   }
   // RoPE tables: cos/sin of pos * base^(-2j/d_axis), computed in double, stored as float2.
+  // Layout [position][pair j]; 3-D: t (frames), h (grid rows), w (grid columns); 1-D: angle
+  // of the frame offset frame*L_f, then of the in-frame token index.
   for (int e = threadIdx.x; e < p.tab_entries; e += kThreads) {
     int pos, j, da;
     if (p.rope_mode == 3) {
@@ -243,6 +260,21 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
     sincospi(turns, &sn, &cs);
     tab[e] = make_float2(static_cast<float>(cs), static_cast<float>(sn));
   }
+  __syncthreads();
+  if (warp == 0) {
+    // compact the live tiles, 32 at a time, keeping their order
+    int base = 0;
+    for (int n0 = 0; n0 < n_tiles; n0 += 32) {
+      const int n = n0 + lane;
+      const uint8_t f = n < n_tiles ? tile_flag[n] : 0;
+      const uint32_t live = __ballot_sync(0xffffffffu, f & 1);
+      if (f & 1)
+        tile_list[base + __popc(live & ((1u << lane) - 1u))] =
+            static_cast<uint16_t>(n | ((f & 2) ? 0x8000 : 0));
+      base += __popc(live);
+    }
+    if (lane == 0) n_live_s = base;
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -250,7 +282,7 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
   const uint32_t tmem = tmem_base_s;
   const unsigned vm = vmask_s;
   const uint64_t deadline = globaltimer() + p.timeout_ns;
-  const int n_tiles = (p.T + BN - 1) / BN;
+  const int n_live = n_live_s;
 
   if (warp >= kProducerWarp) {
     setmaxnreg_dec<72>();
@@ -261,9 +293,9 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
         for (int pp = 0; pp < D / 64; ++pp)
           tma_load_3d(sQ + qt * LY::kTileBytes + pp * 16384, &tm_q, bar(B_QFULL), pp * 64, h,
                       q0 + qt * BM);
-      int j = 0;
-      for (int n = 0; n < n_tiles; ++n) {
-        if (!tile_live(n, vm, p)) continue;
+      int j = 0, last_k = -1, last_v = -1;               // last iterations whose loads went out
+      for (; j < n_live; ++j) {
+        const int n = tile_list[j] & 0x7fff;
         const int st = j & 1;
         const uint32_t par = ((j >> 1) - 1) & 1;
         if (j >= 2 && !mbar_wait(bar(B_KEMPTY + st), par, &ab, deadline, p.status)) break;
@@ -271,23 +303,20 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
         for (int pp = 0; pp < D / 64; ++pp)
           tma_load_3d(sK + st * LY::kTileBytes + pp * 16384, &tm_k, bar(B_KFULL + st), pp * 64,
                       n * BN, h);
+        last_k = j;
         if (j >= 2 && !mbar_wait(bar(B_VEMPTY + st), par, &ab, deadline, p.status)) break;
         mbar_arrive_expect_tx(bar(B_VFULL + st), LY::kTileBytes);
         for (int pp = 0; pp < D / 64; ++pp)
           tma_load_3d(sV + st * LY::kTileBytes + pp * 16384, &tm_v, bar(B_VFULL + st), pp * 64,
                       n * BN, h);
-        ++j;
+        last_v = j;
       }
       if (ab.flag) {     // let copies in flight land before the CTA's shared memory goes away
-        // the last loads issued into stage s belong to iteration j-1-((j-1-s)&1)
         drain_wait(bar(B_QFULL), 0, 100000000ull);
-        for (int s = 0; s < 2; ++s) {
-          const int last = j - 1 - ((j - 1 - s) & 1);
-          if (last >= 0) {
-            drain_wait(bar(B_KFULL + s), (last >> 1) & 1, 100000000ull);
-            drain_wait(bar(B_VFULL + s), (last >> 1) & 1, 100000000ull);
-          }
-        }
+        for (int i = last_k - 1; i <= last_k; ++i)
+          if (i >= 0) drain_wait(bar(B_KFULL + (i & 1)), (i >> 1) & 1, 100000000ull);
+        for (int i = last_v - 1; i <= last_v; ++i)
+          if (i >= 0) drain_wait(bar(B_VFULL + (i & 1)), (i >> 1) & 1, 100000000ull);
       }
     } else if (warp == kMmaWarp && lane == 0) {
       // ---------------------------------------------------------------- MMA issuer
@@ -327,8 +356,8 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
       };
       int j = 0;
       bool prev_partial = false;
-      for (int n = 0; ok && n < n_tiles; ++n) {
-        if (!tile_live(n, vm, p)) continue;
+      for (; ok && j < n_live; ++j) {
+        const bool partial = tile_list[j] >> 15;
         const int st = j & 1;
         if (!mbar_wait(bar(B_KREADY + st), (j >> 1) & 1, &ab, deadline, p.status)) { ok = false; break; }
         tc_fence_after();
@@ -342,8 +371,7 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
         s_mma(1, st);
         umma_commit(bar(B_SFULL + 1));
         umma_commit(bar(B_KEMPTY + st));
-        prev_partial = !tile_full(n, vm, p);
-        ++j;
+        prev_partial = partial;
       }
       if (ok && j >= 1) {
         if (pv_mma(0, j - 1, prev_partial)) {
@@ -366,37 +394,54 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
     if (mbar_wait(bar(B_QFULL), 0, &ab, deadline, p.status)) {
       for (int qt = 0; qt < NQ; ++qt) {
         const int qi = q0 + qt * BM + rt;
-        if (qi < p.L_blk)
-          rotate_row<D>(gb + LY::kQ + qt * LY::kTileBytes, rt, p.q_frame + qi / p.L_f,
-                        qi % p.L_f, false, tab, p);
+        if (qi < p.L_blk) {
+          const int tok = qi % p.L_f;
+          rotate_row<D, RT, RH>(gb + LY::kQ + qt * LY::kTileBytes, rt, p.q_frame + qi / p.L_f,
+                                tok / p.grid_w, tok % p.grid_w, false, tab, p);
+        }
       }
       fence_proxy_async_smem();
       mbar_arrive(bar(B_QREADY));
-      int j = 0;
-      for (int n = 0; n < n_tiles; ++n) {
-        if (!tile_live(n, vm, p)) continue;
+      // position of this thread's key row, advanced incrementally from tile to tile
+      int cur = -2 * BN, s_cur = 0, frame = 0, y = 0, x = 0;   // no previous row yet
+      for (int j = 0; j < n_live; ++j) {
+        const uint16_t te = tile_list[j];
+        const int n = te & 0x7fff;
+        const bool partial = te >> 15;
         const int st = j & 1;
         if (!mbar_wait(bar(B_KFULL + st), (j >> 1) & 1, &ab, deadline, p.status)) break;
         const int row = n * BN + rt;
         bool empty = false;
         if (row < p.T) {
-          const int s = slot_of(row, p);
-          const int u = row - p.slot_start[s];
-          empty = !((vm >> s) & 1u);
-          rotate_row<D>(gb + LY::kK + st * LY::kTileBytes, rt, p.slot_frame[s] + u / p.L_f,
-                        u % p.L_f, empty, tab, p);
+          if (row == cur + BN && row < p.slot_start[s_cur + 1]) {
+            x += p.step_x;                       // one tile further in the same slot
+            y += p.step_y;
+            if (x >= p.grid_w) { x -= p.grid_w; ++y; }
+            while (y >= p.grid_h) { y -= p.grid_h; ++frame; }
+          } else {
+            s_cur = slot_of(row, p);
+            const int u = row - p.slot_start[s_cur];
+            const int tok = u % p.L_f;
+            frame = p.slot_frame[s_cur] + u / p.L_f;
+            y = tok / p.grid_w;
+            x = tok - y * p.grid_w;
+          }
+          cur = row;
+          empty = !((vm >> s_cur) & 1u);
+          rotate_row<D, RT, RH>(gb + LY::kK + st * LY::kTileBytes, rt, frame, y, x, empty, tab,
+                                p);
         }
         fence_proxy_async_smem();
         mbar_arrive(bar(B_KREADY + st));
-        if (!tile_full(n, vm, p)) {
+        if (partial) {
           // boundary tile: empty-slot rows of V may hold anything; P is 0 there, but 0 * NaN
           // is not, so zero them before the P.V MMA reads the tile
           if (!mbar_wait(bar(B_VFULL + st), (j >> 1) & 1, &ab, deadline, p.status)) break;
-          if (empty) rotate_row<D>(gb + LY::kV + st * LY::kTileBytes, rt, 0, 0, true, tab, p);
+          if (empty) rotate_row<D, RT, RH>(gb + LY::kV + st * LY::kTileBytes, rt, 0, 0, 0, true,
+                                           tab, p);
           fence_proxy_async_smem();
           mbar_arrive(bar(B_VFIX + st));
         }
-        ++j;
       }
     }
   } else {
@@ -411,8 +456,9 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
     float m = -INFINITY, l = 0.f;
     int j = 0;
     bool ok = true;
-    for (int n = 0; n < n_tiles; ++n) {
-      if (!tile_live(n, vm, p)) continue;
+    for (; j < n_live; ++j) {
+      const uint16_t te = tile_list[j];
+      const int n = te & 0x7fff;
       ok = mbar_wait(bar(B_SFULL + qt), j & 1, &ab, deadline, p.status);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }   // tcgen05.ld is warp-collective
       tc_fence_after();
@@ -422,7 +468,7 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
       tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
       tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
       tmem_wait_ld();
-      if (!tile_full(n, vm, p)) {
+      if (te >> 15) {
         // columns of empty slots and past the end of the cache: 4 mask words, built per slot
         const int lo = n * BN;
         uint32_t mw[4] = {~0u, ~0u, ~0u, ~0u};
@@ -449,12 +495,17 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
         for (int c = 0; c < 128; ++c)
           if (!((mw[c >> 5] >> (c & 31)) & 1u)) s[c] = __float_as_uint(-INFINITY);
       }
-      // row max of the raw scores (scaling by a positive constant keeps the argmax)
-      float mt = fmax3(__uint_as_float(s[0]), __uint_as_float(s[1]), __uint_as_float(s[2]));
+      // row max of the raw scores (scaling by a positive constant keeps the argmax); eight
+      // independent partial maxima keep the dependency chains short
+      float mx[8];
 #pragma unroll
-      for (int c = 3; c < 127; c += 2)
-        mt = fmax3(mt, __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
-      mt = fmaxf(mt, __uint_as_float(s[127])) * p.scale_log2;
+      for (int a = 0; a < 8; ++a) mx[a] = __uint_as_float(s[a]);
+#pragma unroll
+      for (int c = 8; c < 128; c += 8)
+#pragma unroll
+        for (int a = 0; a < 8; ++a) mx[a] = fmaxf(mx[a], __uint_as_float(s[c + a]));
+      const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                             fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * p.scale_log2;
       float alpha = 1.f;
       bool rescale = false;
       if (j == 0) {
@@ -467,7 +518,8 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
       // P = 2^(s*scale - m) as bf16 pairs into the S columns (A operand of the P.V MMA):
       // 32 scores -> 16 packed words -> one 16-column TMEM store
       const float2 negm = make_float2(-m, -m);
-      float2 sum2 = make_float2(0.f, 0.f);
+      float2 sum2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                        make_float2(0.f, 0.f)};               // independent partial sums
 #pragma unroll
       for (int ch = 0; ch < 4; ++ch) {
         uint32_t pk[16];
@@ -477,12 +529,14 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
           const float2 e2 = ffma2(make_float2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])),
                                   scale2, negm);
           const float2 pr = make_float2(ex2(e2.x), ex2(e2.y));
-          sum2 = fadd2(sum2, pr);
+          sum2[i & 3] = fadd2(sum2[i & 3], pr);
           pk[i] = pack_bf16(pr.x, pr.y);
         }
         tmem_st16(tS + ch * 16, pk);
       }
-      l = l * alpha + (sum2.x + sum2.y);
+      const float2 s01 = fadd2(sum2[0], sum2[1]), s23 = fadd2(sum2[2], sum2[3]);
+      const float2 s4 = fadd2(s01, s23);
+      l = l * alpha + (s4.x + s4.y);
       if (__any_sync(0xffffffffu, rescale)) {   // rows that keep their max scale by alpha = 1
         // O_qt holds every P.V up to tile j-1: the S(j) commit completed after them
 #pragma unroll 1
@@ -498,7 +552,6 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(B_PFULL + qt));
-      ++j;
     }
     // epilogue: O / l -> bf16, one 2*D-byte row per thread
     const int qi = q0 + qt * BM + t;
@@ -588,7 +641,7 @@ static int make_map(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, 
   return PRSINK_OK;
 }
 
-template <int D>
+template <int D, int RT, int RH>
 static int launch(const prsink_layout* L, const Geometry& g, const void* q, const void* k,
                   const void* v, Params& p, cudaStream_t st) {
   CUtensorMap mq, mk, mv;
@@ -604,13 +657,13 @@ static int launch(const prsink_layout* L, const Geometry& g, const void* q, cons
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) dev = 0;
   if (attr_bytes[dev] < smem) {
-    if (cudaFuncSetAttribute(prsink_attention_kernel<D>,
+    if (cudaFuncSetAttribute(prsink_attention_kernel<D, RT, RH>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return check_launch("prsink_attention: shared memory attribute");
     attr_bytes[dev] = smem;
   }
   dim3 grid((g.L_blk + NQ * BM - 1) / (NQ * BM), L->n_heads);
-  prsink_attention_kernel<D><<<grid, kThreads, smem, st>>>(mq, mk, mv, p);
+  prsink_attention_kernel<D, RT, RH><<<grid, kThreads, smem, st>>>(mq, mk, mv, p);
   count_launch();
   return check_launch("prsink_attention");
 }
@@ -681,6 +734,12 @@ extern "C" int prsink_attention(const prsink_layout* layout, const void* q, cons
     p.tab_w_off = p.tab_h_off + p.L_f * (D / 2);
     p.tab_entries = p.tab_w_off;
   }
+  p.step_y = BN / layout->grid_w;
+  p.step_x = BN % layout->grid_w;
+  if ((g.T + BN - 1) / BN > kMaxTiles) {
+    set_error("prsink_attention: %lld keys exceed the %d-tile limit", g.T, kMaxTiles);
+    return PRSINK_ERR_UNSUPPORTED;
+  }
   if (p.tab_entries * 8 > kTableMaxBytes) {
     set_error("prsink_attention: RoPE tables need %d bytes of shared memory (max %d)",
               p.tab_entries * 8, kTableMaxBytes);
@@ -696,6 +755,8 @@ extern "C" int prsink_attention(const prsink_layout* layout, const void* q, cons
   if (!p.status) return PRSINK_ERR_LAUNCH;
   if (g.L_blk == 0) return PRSINK_OK;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  return D == 128 ? launch<128>(layout, g, q, k_cache, v_cache, p, st)
-                  : launch<64>(layout, g, q, k_cache, v_cache, p, st);
+  if (D == 128 && p.rope_mode == 3 && p.rd[0] == 22 && p.rd[1] == 21)   // 44/42/42 split
+    return launch<128, 22, 21>(layout, g, q, k_cache, v_cache, p, st);
+  return D == 128 ? launch<128, 0, 0>(layout, g, q, k_cache, v_cache, p, st)
+                  : launch<64, 0, 0>(layout, g, q, k_cache, v_cache, p, st);
 }

@@ -12,6 +12,7 @@ import oracle
 import pose_retrieved_kv_b200 as P
 import synth
 from tests._gpu import (LSE_MAX_ABS, attention_inputs, check_attention, f64, need_gpu)
+from tests._probe import probe_inputs
 
 pytestmark = pytest.mark.gpu
 
@@ -62,6 +63,46 @@ def test_small_3d_every_element(ci, b, mask):
     ref, ref_lse = oracle.attention(cfg, f64(q), f64(k), f64(v))
     check_attention(got, ref, f"3d cfg{ci} b={b}")
     assert np.abs(lse - ref_lse).max() <= LSE_MAX_ABS
+
+
+@pytest.mark.parametrize("S,sign", [(5.0, -1.0), (60.0, -1.0), (900.0, -1.0), (60.0, 1.0),
+                                    (900.0, 1.0)])
+def test_scores_far_from_zero(S, sign):
+    """Every score about sign * S (tests/_probe.py): the running max must follow rows whose
+    scores are all large negative or large positive (a max stuck at 0 underflows every weight
+    and returns LSE = -inf, O = 0).  The kernel rounds rotated q and k to bf16, so score errors
+    grow like 2^-9 * |score|: the bounds scale with S."""
+    need_gpu()
+    cfg = synth.preset("tiny", block_index=7, valid_mask=0xFF)
+    q, k, v = probe_inputs(cfg, S, seed=3, sign=sign)
+    got, lse = _run(cfg, q, k, v)
+    ref, ref_lse = oracle.attention(cfg, f64(q), f64(k), f64(v))
+    assert np.all(np.isfinite(lse))
+    assert np.abs(lse - ref_lse).max() <= 2e-2 + 2.5e-3 * S
+    assert np.abs(got - ref).max() <= 2e-2 + 1e-4 * S
+    assert np.abs(got).max() > 0.1 * np.abs(ref).max()        # not an all-zero output
+
+
+@pytest.mark.parametrize("name,slot,gain", [("tiny", 5, 6.0), ("480x480", 5, 5.0),
+                                            ("480x480", 0, 5.0)])
+def test_max_growing_or_shrinking_across_tiles(name, slot, gain):
+    """Keys of one slot scaled by `gain`: when it is the last slot the row max grows by far
+    more than 2^8 between key tiles, so the output accumulator is rescaled mid-row; when it
+    is the ref slot (first tiles) later tiles sit far below the max instead."""
+    need_gpu()
+    cfg = synth.preset(name, block_index=1000, valid_mask=0xFF)
+    if name != "tiny":
+        cfg = dict(cfg, n_heads=4)
+    q, k, v = attention_inputs(cfg, seed=13)
+    a, e = oracle.slot_ranges(cfg)[slot]
+    k = k.clone()
+    k[:, a:e] = (k[:, a:e].float() * gain).to(torch.bfloat16)
+    got, lse = _run(cfg, q, k, v)
+    s = oracle.layout_sizes(cfg)
+    rows = _sample_rows(s["L_blk"], 9) if name != "tiny" else np.arange(s["L_blk"])
+    ref, ref_lse = oracle.attention(cfg, f64(q), f64(k), f64(v), rows=rows)
+    check_attention(got[rows], ref, f"{name} slot {slot} x{gain}")
+    assert np.abs(lse[:, rows] - ref_lse).max() <= LSE_MAX_ABS * gain
 
 
 def test_no_valid_key_gives_zeros():
@@ -128,3 +169,34 @@ def test_full_size_early_block():
     rows = _sample_rows(2700, 8)
     ref, _ = oracle.attention(cfg, f64(q), f64(k), f64(v), rows=rows, heads=[0, 17, 39])
     check_attention(got[rows][:, [0, 17, 39]], ref, "480x480 b=1")
+
+
+# Position probe (tests/_probe.py): correctly rotated keys all score -S; a key rotated at a
+# wrong position takes over the output (a one-column shift of one key moves the output by
+# 0.36 at the tiny layout and 2.9 at 480x480).  Legitimate rounding (bf16 rotated q and k, bf16
+# P) stays below 0.015 and 0.006 on these inputs, so the bounds below separate the two.
+PROBES = [
+    ("tiny", 300.0, 1, 7, 0xFF, 0.05),
+    ("tiny", 300.0, 1, 1, 0b011011, 0.05),
+    ("480x480", 1000.0, 2, 1000, 0xFF, 0.03),
+    ("480x480", 1000.0, 2, 4, 0b0111011, 0.03),
+    ("384x672_r4", 1000.0, 2, 1001, 0xFF, 0.03),
+    ("672x384", 1000.0, 2, 999, 0xFF, 0.03),
+]
+
+
+@pytest.mark.parametrize("name,S,H,b,mask,bound", PROBES)
+def test_every_key_rotated_at_its_position(name, S, H, b, mask, bound):
+    need_gpu()
+    cfg = synth.preset(name, block_index=b, valid_mask=mask, n_heads=H)
+    q, k, v = probe_inputs(cfg, S)
+    got, lse = _run(cfg, q, k, v)
+    s = oracle.layout_sizes(cfg)
+    rows = np.unique(np.concatenate([np.arange(0, s["L_blk"], 37), [s["L_blk"] - 1]]))
+    ref, ref_lse = oracle.attention(cfg, f64(q), f64(k), f64(v), rows=rows)
+    err = np.abs(got[rows] - ref)
+    assert err.max() <= bound, f"{name} b={b}: max {err.max():.3e}"
+    # every score is about -S here: the running max must follow negative scores (an output of
+    # zeros would also be within `bound` at large T; the LSE is not)
+    assert np.all(np.isfinite(lse[:, rows]))
+    assert np.abs(lse[:, rows] - ref_lse).max() <= 1e-3 * S, f"{name}: LSE"

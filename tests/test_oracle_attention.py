@@ -203,3 +203,31 @@ def test_rows_and_heads_subsets_match_full():
     sub, lse_s = oracle.attention(cfg, q, k, v, rows=rows, heads=[1])
     assert np.max(np.abs(sub[:, 0] - full[rows, 1])) <= 1e-14
     assert np.max(np.abs(lse_s[0] - lse[1, rows])) <= 1e-14
+
+
+def test_position_probe_catches_one_misplaced_key(monkeypatch):
+    """The adversarial probe of the GPU position tests is sensitive: moving ONE key of the
+    cache one grid column (3-D) or one token (1-D) changes the output far beyond the
+    attention tolerance."""
+    import oracle.prsink_oracle as po
+    from tests._probe import probe_inputs
+    for name, S, H in [("tiny", 300.0, 1), ("480x480", 1000.0, 1)]:
+        cfg = synth.preset(name, block_index=1000, valid_mask=0xFF, n_heads=H)
+        q, k, v = (t.double().numpy() for t in probe_inputs(cfg, S))
+        rows = np.arange(0, oracle.layout_sizes(cfg)["L_blk"], 97)
+        good, _ = oracle.attention(cfg, q, k, v, rows=rows)
+        orig = po.key_positions
+
+        def shifted(c):
+            pos, valid = orig(c)
+            pos = pos.copy()
+            if c["rope_mode"] == 3:
+                pos[127, 2] += 1
+            else:
+                pos[127] += 1
+            return pos, valid
+
+        monkeypatch.setattr(po, "key_positions", shifted)
+        bad, _ = oracle.attention(cfg, q, k, v, rows=rows)
+        monkeypatch.setattr(po, "key_positions", orig)
+        assert np.abs(bad - good).max() > 0.25, name
