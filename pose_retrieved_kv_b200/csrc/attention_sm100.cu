@@ -4,8 +4,8 @@
 //
 // One CTA computes 256 queries (two 128-row tiles Q0, Q1) of one head, ping-ponging the two
 // tiles so that the tensor core works on one tile while the other tile's softmax runs.
-// Warp roles (512 threads; setmaxnreg gives the softmax warps 192 registers, the rotation
-// warps 56 and the producer / MMA warps 72):
+// Warp roles (512 threads; setmaxnreg gives the softmax warps 184 registers, the rotation
+// warps 64 and the producer / MMA warps 80):
 //   warps 0-3   softmax of Q0, warps 4-7 softmax of Q1: thread t owns query row t (TMEM lane
 //               t); it reads S from TMEM, keeps the running max and sum, writes P as bf16 back
 //               into the S columns (the A operand of the P.V MMA), rescales O in TMEM when the
@@ -124,6 +124,103 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64
     if (globaltimer() > dl) break;
 }
 
+// Rotation of two adjacent pairs of one axis at once in the two lanes of the packed fp32 FMA:
+// words a, b hold (x0, x1) of pairs P and P+1 as bf16 pairs; cs = (cos_P, cos_P+1, sin_P,
+// sin_P+1), ns = (-sin_P, -sin_P+1).  y0 = x0 cos - x1 sin, y1 = x0 sin + x1 cos.
+__device__ __forceinline__ void rot_pair2(uint32_t& a, uint32_t& b, float4 cs, float2 ns) {
+  const float2 x0 = make_float2(__uint_as_float(a << 16), __uint_as_float(b << 16));
+  const float2 x1 = make_float2(__uint_as_float(a & 0xFFFF0000u), __uint_as_float(b & 0xFFFF0000u));
+  const float2 c = make_float2(cs.x, cs.y);
+  const float2 y0 = ffma2(x1, ns, fmul2(x0, c));
+  const float2 y1 = ffma2(x1, c, fmul2(x0, make_float2(cs.z, cs.w)));
+  a = pack_bf16(y0.x, y1.x);
+  b = pack_bf16(y0.y, y1.y);
+}
+
+__device__ __forceinline__ void rot_pair1(uint32_t& a, float c, float sn) {
+  const float x0 = __uint_as_float(a << 16), x1 = __uint_as_float(a & 0xFFFF0000u);
+  a = pack_bf16(x0 * c - x1 * sn, x0 * sn + x1 * c);
+}
+
+// Grouped tables of the compile-time split (3-D RoPE, d = 128): for every axis and position,
+// records of two consecutive pairs: float4 (cos, cos', sin, sin') and float2 (-sin, -sin').
+template <int RT, int RH>
+struct Groups {
+  static constexpr int RW = 64 - RT - RH;
+  static constexpr int GT = (RT + 1) / 2, GH = (RH + 1) / 2, GW = (RW + 1) / 2;
+};
+
+__device__ __forceinline__ uint4 lds_u4(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a) : "memory");
+  return v;
+}
+__device__ __forceinline__ void sts_u4(uint32_t a, uint4 v) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
+               :: "r"(a), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
+}
+// Loads of the RoPE tables, which do not change after the prologue: free to be scheduled.
+__device__ __forceinline__ float4 lds_f4(uint32_t a) {
+  float4 v;
+  asm("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+      : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ float2 lds_f2(uint32_t a) {
+  float2 v;
+  asm("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(a));
+  return v;
+}
+
+// Rotate one row (128 bf16, two 128-byte swizzled panels at shared address `tile`) at
+// (frame, y, x) with the grouped tables (shared addresses `cs`, `ns`).  Pair P lives in 32-bit
+// word P of the row.  Groups of two pairs always start at an even word: t pairs (0,1)..(20,21);
+// h pairs (22,23)..(40,41) then 42 alone; w pair 43 alone then (44,45)..(62,63).  So no group
+// crosses a 16-byte chunk and the row is processed chunk by chunk (few live registers).
+template <int RT, int RH>
+__device__ __forceinline__ void rotate_row_grouped(uint32_t tile, int r, int frame, int y, int x,
+                                                   bool zero, uint32_t cs, uint32_t ns,
+                                                   const Params& p) {
+  static_assert(RT == 22 && RH == 21, "the grouping is written for the 44/42/42 split");
+  using G = Groups<RT, RH>;
+  const int offH = p.n_frames * G::GT, offW = offH + p.grid_h * G::GH;
+  const uint32_t csT = cs + frame * G::GT * 16, nsT = ns + frame * G::GT * 8;
+  const uint32_t csH = cs + (offH + y * G::GH) * 16, nsH = ns + (offH + y * G::GH) * 8;
+  const uint32_t csW = cs + (offW + x * G::GW) * 16, nsW = ns + (offW + x * G::GW) * 8;
+  const uint32_t row = tile + r * 128;
+  const uint32_t sw = (r & 7) << 4;
+#pragma unroll
+  for (int c = 0; c < 16; ++c) {
+    const uint32_t addr = row + (c >> 3) * 16384 + (((c & 7) << 4) ^ sw);
+    if (zero) {
+      sts_u4(addr, make_uint4(0, 0, 0, 0));
+      continue;
+    }
+    const uint4 v = lds_u4(addr);
+    uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; i += 2) {
+      const int P = 4 * c + i;                         // even word: a group or singles
+      if (P < RT) {
+        rot_pair2(w[i], w[i + 1], lds_f4(csT + (P / 2) * 16), lds_f2(nsT + (P / 2) * 8));
+      } else if (P + 1 < RT + RH) {
+        const int j = P - RT;
+        rot_pair2(w[i], w[i + 1], lds_f4(csH + (j / 2) * 16), lds_f2(nsH + (j / 2) * 8));
+      } else if (P < RT + RH) {                        // words 42 (h, last) and 43 (w, first)
+        const float4 h4 = lds_f4(csH + ((RH - 1) / 2) * 16);
+        rot_pair1(w[i], h4.x, h4.z);
+        const float4 w4 = lds_f4(csW);
+        rot_pair1(w[i + 1], w4.x, w4.z);
+      } else {
+        const int g = (P - RT - RH + 1) / 2;           // w record 1.. holds pairs (2g-1, 2g)
+        rot_pair2(w[i], w[i + 1], lds_f4(csW + g * 16), lds_f2(nsW + g * 8));
+      }
+    }
+    sts_u4(addr, make_uint4(w[0], w[1], w[2], w[3]));
+  }
+}
+
 // Rotate one 128-byte-swizzled row (D bf16 over D/64 panels) in place at position
 // (frame, tok); or zero it when `zero` is set.  RT, RH: pairs of the t and h axes when known
 // at compile time (3-D RoPE), 0 to read the split from the parameters.
@@ -240,9 +337,37 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
     tmem_relinquish();
   }
   // RoPE tables: cos/sin of pos * base^(-2j/d_axis), computed in double, stored as float2.
+  float4* gcs = reinterpret_cast<float4*>(gb + LY::kTab);   // grouped tables (RT > 0)
+  using GR = Groups<(RT > 0 ? RT : 22), (RT > 0 ? RH : 21)>;
+  const int g_count = p.n_frames * GR::GT + p.grid_h * GR::GH + p.grid_w * GR::GW;
+  float2* gns = reinterpret_cast<float2*>(gcs + g_count);
+  if constexpr (RT > 0) {
+    const int offH = p.n_frames * GR::GT, offW = offH + p.grid_h * GR::GH;
+    for (int e = threadIdx.x; e < g_count; e += kThreads) {
+      int pos, g, na;
+      if (e < offH) { pos = e / GR::GT; g = e % GR::GT; na = RT; }
+      else if (e < offW) { pos = (e - offH) / GR::GH; g = (e - offH) % GR::GH; na = RH; }
+      else { pos = (e - offW) / GR::GW; g = (e - offW) % GR::GW; na = GR::RW; }
+      double sn[2] = {0.0, 0.0}, cs[2] = {1.0, 1.0};
+      const bool w_axis = e >= offW;
+      for (int l = 0; l < 2; ++l) {
+        // t, h: record g holds pairs (2g, 2g+1); w: record 0 holds pair 0, record g >= 1
+        // holds pairs (2g-1, 2g)
+        const int jj = w_axis ? (g == 0 ? (l == 0 ? 0 : na) : 2 * g - 1 + l) : 2 * g + l;
+        if (jj < na) {
+          const double turns = static_cast<double>(pos) *
+                               exp2(-(2.0 * jj / (2 * na)) * p.log2_base) * 0.31830988618379067154;
+          sincospi(turns, &sn[l], &cs[l]);
+        }
+      }
+      gcs[e] = make_float4(static_cast<float>(cs[0]), static_cast<float>(cs[1]),
+                           static_cast<float>(sn[0]), static_cast<float>(sn[1]));
+      gns[e] = make_float2(-static_cast<float>(sn[0]), -static_cast<float>(sn[1]));
+    }
+  }
   // Layout [position][pair j]; 3-D: t (frames), h (grid rows), w (grid columns); 1-D: angle
   // of the frame offset frame*L_f, then of the in-frame token index.
-  for (int e = threadIdx.x; e < p.tab_entries; e += kThreads) {
+  for (int e = threadIdx.x; RT == 0 && e < p.tab_entries; e += kThreads) {
     int pos, j, da;
     if (p.rope_mode == 3) {
       if (e < p.tab_h_off) { pos = e / p.rd[0]; j = e % p.rd[0]; da = 2 * p.rd[0]; }
@@ -285,7 +410,7 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
   const int n_live = n_live_s;
 
   if (warp >= kProducerWarp) {
-    setmaxnreg_dec<72>();
+    setmaxnreg_dec<80>();
     if (warp == kProducerWarp && lane == 0) {
       // ---------------------------------------------------------------- TMA producer
       mbar_arrive_expect_tx(bar(B_QFULL), NQ * LY::kTileBytes);
@@ -359,9 +484,10 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
       for (; ok && j < n_live; ++j) {
         const bool partial = tile_list[j] >> 15;
         const int st = j & 1;
+        // P0(j-1).V(j-1) does not need K(j): issue it before waiting for the rotation
+        if (j >= 1 && !pv_mma(0, j - 1, prev_partial)) { ok = false; break; }
         if (!mbar_wait(bar(B_KREADY + st), (j >> 1) & 1, &ab, deadline, p.status)) { ok = false; break; }
         tc_fence_after();
-        if (j >= 1 && !pv_mma(0, j - 1, prev_partial)) { ok = false; break; }
         s_mma(0, st);
         umma_commit(bar(B_SFULL + 0));
         if (j >= 1) {
@@ -389,15 +515,20 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
     }
   } else if (warp >= kRotWarp0) {
     // ------------------------------------------------------------------ rotation
-    setmaxnreg_dec<56>();
+    setmaxnreg_dec<64>();
     const int rt = threadIdx.x - kRotWarp0 * 32;          // row of the tile, 0..127
     if (mbar_wait(bar(B_QFULL), 0, &ab, deadline, p.status)) {
       for (int qt = 0; qt < NQ; ++qt) {
         const int qi = q0 + qt * BM + rt;
         if (qi < p.L_blk) {
           const int tok = qi % p.L_f;
-          rotate_row<D, RT, RH>(gb + LY::kQ + qt * LY::kTileBytes, rt, p.q_frame + qi / p.L_f,
-                                tok / p.grid_w, tok % p.grid_w, false, tab, p);
+          if constexpr (RT > 0)
+            rotate_row_grouped<RT, RH>(sQ + qt * LY::kTileBytes, rt, p.q_frame + qi / p.L_f,
+                                       tok / p.grid_w, tok % p.grid_w, false, smem_u32(gcs),
+                                       smem_u32(gns), p);
+          else
+            rotate_row<D, RT, RH>(gb + LY::kQ + qt * LY::kTileBytes, rt, p.q_frame + qi / p.L_f,
+                                  tok / p.grid_w, tok % p.grid_w, false, tab, p);
         }
       }
       fence_proxy_async_smem();
@@ -428,8 +559,12 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
           }
           cur = row;
           empty = !((vm >> s_cur) & 1u);
-          rotate_row<D, RT, RH>(gb + LY::kK + st * LY::kTileBytes, rt, frame, y, x, empty, tab,
-                                p);
+          if constexpr (RT > 0)
+            rotate_row_grouped<RT, RH>(sK + st * LY::kTileBytes, rt, frame, y, x, empty,
+                                       smem_u32(gcs), smem_u32(gns), p);
+          else
+            rotate_row<D, RT, RH>(gb + LY::kK + st * LY::kTileBytes, rt, frame, y, x, empty, tab,
+                                  p);
         }
         fence_proxy_async_smem();
         mbar_arrive(bar(B_KREADY + st));
@@ -446,7 +581,7 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
     }
   } else {
     // ------------------------------------------------------------------ softmax (warps 0-7)
-    setmaxnreg_inc<192>();
+    setmaxnreg_inc<184>();
     const int qt = warp >> 2;                             // query tile of this warpgroup
     const int t = threadIdx.x & (BM - 1);                 // query row = TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
@@ -649,7 +784,14 @@ static int launch(const prsink_layout* L, const Geometry& g, const void* q, cons
   if (!rc) rc = make_map(&mk, k, D, g.T, L->n_heads, 2ull * D, 2ull * D * g.T, BN, 1);
   if (!rc) rc = make_map(&mv, v, D, g.T, L->n_heads, 2ull * D, 2ull * D * g.T, BN, 1);
   if (rc) return rc;
-  const int tab_bytes = p.tab_entries * 8;
+  using GR = Groups<22, 21>;
+  const int tab_bytes = RT > 0 ? (p.n_frames * GR::GT + L->grid_h * GR::GH + L->grid_w * GR::GW) * 24
+                               : p.tab_entries * 8;
+  if (tab_bytes > kTableMaxBytes) {
+    set_error("prsink_attention: RoPE tables need %d bytes of shared memory (max %d)", tab_bytes,
+              kTableMaxBytes);
+    return PRSINK_ERR_UNSUPPORTED;
+  }
   int smem = Layout<D>::kTab + tab_bytes + 1024;
   if (smem < 120 * 1024) smem = 120 * 1024;     // one CTA per SM (it holds all 512 TMEM columns)
   static int attr_bytes[64] = {0};      // largest size already allowed, per device

@@ -101,8 +101,18 @@ def test_max_growing_or_shrinking_across_tiles(name, slot, gain):
     s = oracle.layout_sizes(cfg)
     rows = _sample_rows(s["L_blk"], 9) if name != "tiny" else np.arange(s["L_blk"])
     ref, ref_lse = oracle.attention(cfg, f64(q), f64(k), f64(v), rows=rows)
-    check_attention(got[rows], ref, f"{name} slot {slot} x{gain}")
-    assert np.abs(lse[:, rows] - ref_lse).max() <= LSE_MAX_ABS * gain
+    # bf16 rounding of the rotated q and k moves a logit by ~2^-9 |logit|; with logits up to
+    # s_max (>> the ~4 of N(0,1) inputs) the softmax is sharp, so the bound grows with s_max
+    kpos, _ = oracle.key_positions(cfg)
+    qpos = oracle.query_positions(cfg)
+    s_max = max(np.abs(oracle.rope_rotate(cfg, f64(q)[rows, h], qpos[rows])
+                       @ oracle.rope_rotate(cfg, f64(k)[h], kpos).T).max()
+                for h in range(cfg["n_heads"])) / np.sqrt(cfg["head_dim"])
+    bound = 2e-2 * max(1.0, s_max / 8.0)
+    err = np.abs(got[rows] - ref)
+    assert np.all(np.isfinite(got)) and err.max() <= bound, (err.max(), bound)
+    assert err.mean() <= 2e-3 * max(1.0, s_max / 8.0)
+    assert np.abs(lse[:, rows] - ref_lse).max() <= LSE_MAX_ABS * max(1.0, s_max / 8.0)
 
 
 def test_no_valid_key_gives_zeros():
