@@ -350,6 +350,7 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
       else { pos = (e - offW) / GR::GW; g = (e - offW) % GR::GW; na = GR::RW; }
       double sn[2] = {0.0, 0.0}, cs[2] = {1.0, 1.0};
       const bool w_axis = e >= offW;
+#pragma unroll
       for (int l = 0; l < 2; ++l) {
         // t, h: record g holds pairs (2g, 2g+1); w: record 0 holds pair 0, record g >= 1
         // holds pairs (2g-1, 2g)
@@ -448,15 +449,14 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
       bool ok = mbar_wait(bar(B_QREADY), 0, &ab, deadline, p.status);
       tc_fence_after();
       int fix0 = 0, fix1 = 0;                              // boundary tiles seen per stage
+      // base descriptors, computed once: Q0, Q1, the two K stages and the two V stages
+      const uint64_t dq0 = sdesc_sw128(sQ, 16, 1024), dq1 = sdesc_sw128(sQ + LY::kTileBytes, 16, 1024);
+      const uint64_t dk0 = sdesc_sw128(sK, 16, 1024), dk1 = sdesc_sw128(sK + LY::kTileBytes, 16, 1024);
+      const uint64_t dv0 = sdesc_sw128(sV, 16384, 1024), dv1 = sdesc_sw128(sV + LY::kTileBytes, 16384, 1024);
       auto s_mma = [&](int qt, int st) {
-        const uint32_t q_base = sQ + qt * LY::kTileBytes;
-        const uint32_t k_base = sK + st * LY::kTileBytes;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          umma_ss(tmem + LY::col_s(qt), sdesc_sw128(q_base + off, 16, 1024),
-                  sdesc_sw128(k_base + off, 16, 1024), LY::kIdescS, kk > 0 ? 1u : 0u);
-        }
+        const uint64_t a = qt ? dq1 : dq0, b = st ? dk1 : dk0;
+        if constexpr (D == 128) umma_ss_k128(tmem + LY::col_s(qt), a, b, LY::kIdescS);
+        else umma_ss_k64(tmem + LY::col_s(qt), a, b, LY::kIdescS);
       };
       // O_qt (+)= P_qt(i) V(i); V(i) must have landed (and been fixed up in boundary tiles)
       auto pv_mma = [&](int qt, int i, bool partial) -> bool {
@@ -471,12 +471,8 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
         }
         if (!mbar_wait(bar(B_PFULL + qt), i & 1, &ab, deadline, p.status)) return false;
         tc_fence_after();
-        const uint32_t v_base = sV + st * LY::kTileBytes;
-#pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk)
-          umma_ts(tmem + LY::col_o(qt), tmem + LY::col_s(qt) + kk * 8,
-                  sdesc_sw128(v_base + kk * 2048, 16384, 1024), LY::kIdescPV,
-                  (i > 0 || kk > 0) ? 1u : 0u);
+        umma_ts_pv128(tmem + LY::col_o(qt), tmem + LY::col_s(qt), st ? dv1 : dv0, LY::kIdescPV,
+                      i > 0 ? 1u : 0u);
         return true;
       };
       int j = 0;
