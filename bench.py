@@ -418,7 +418,7 @@ def oracle_sample_seconds_per_layer_block(cfg, heads: int, seed: int = 0):
 
 
 def cpu_baseline(args, cfg):
-    heads = args.cpu_heads
+    heads = args.baseline_heads
     per_lb, el = oracle_sample_seconds_per_layer_block(cfg, heads)
     return {"value": round(1.0 / per_lb, 6), "unit": UNIT, "cores": _cores(), "kind": "oracle",
             "sample": f"{heads} of {cfg['n_heads']} heads, 1 pass (append + attention, all "
@@ -473,7 +473,10 @@ def main():
     ap.add_argument("--config", default="480x480")
     ap.add_argument("--layers", type=int, default=40)
     ap.add_argument("--pool", type=int, default=8)
-    ap.add_argument("--cpu-heads", type=int, default=4)
+    ap.add_argument("--cpu-heads", type=int, default=4,
+                    help="heads per step of the CPU oracle in --impl reference")
+    ap.add_argument("--baseline-heads", type=int, default=40,
+                    help="heads of the CPU oracle sample in the cpu_baseline leg (~10-30 s)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only", choices=["attention", "append"], default=None,
