@@ -50,6 +50,32 @@ def _peaks():
     return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
 
 
+def _profiled_traffic(src_rel: str, profile_rel: str):
+    """DRAM bytes per launch (read + write) recorded from an ncu capture in ``profiles/``, or
+    None when the kernel source has changed since that capture (sha256 mismatch)."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, src_rel), "rb") as f:
+            digest = hashlib.sha256(f.read()).hexdigest()
+        with open(os.path.join(ROOT, profile_rel)) as f:
+            text = f.read()
+    except OSError:
+        return None
+    rec_hash = rec_bytes = None
+    for line in text.splitlines():
+        if line.startswith("kernel source sha256:"):
+            rec_hash = line.split(":", 1)[1].strip()
+        elif line.startswith("DRAM bytes per launch (read + write):"):
+            rec_bytes = int(line.split(":", 1)[1].strip())
+    return rec_bytes if rec_hash == digest else None
+
+
+ATTN_SRC = "pose_retrieved_kv_b200/csrc/attention_sm100.cu"
+ATTN_PROFILE = "profiles/attention_480x480.md"
+APPEND_SRC = "pose_retrieved_kv_b200/csrc/kv_copy.cu"
+APPEND_PROFILE = "profiles/append_480x480.md"
+
+
 class ClockSampler:
     """nvidia-smi clock / throttle sampling while the timed region runs."""
 
@@ -223,7 +249,11 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                       "frac_of_bf16_peak": round(achieved / peak, 4),
                       "launches_timed": len(attn_ms)},
         "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
-                     "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": None,
+                     "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                     "traffic": (_profiled_traffic(ATTN_SRC, ATTN_PROFILE)
+                                 if args.config == "480x480" else None),
+                     "traffic_source": f"{ATTN_PROFILE}: ncu dram__bytes_read.sum + "
+                                       "dram__bytes_write.sum, bytes per launch",
                      "peak_source": f"{peaks['source']} bf16_tflops_sustained"},
         "gpu_launches": int(launches),
         "clocks": clk,
@@ -237,7 +267,10 @@ def run_ours(args, rank: int, world: int, local_rank: int):
 
 def run_kernel_only(args, local_rank: int):
     """Time one kernel alone (``--only attention|append``) at the workload's sizes: W warm-up
-    launches, then K launches on fresh buffers (a rotating set larger than L2)."""
+    launches, then K launches on rotating buffers (a set larger than L2).  A device-side sleep
+    is queued ahead of the timed launches so that the host has enqueued them all before the
+    first one starts: each event pair then brackets one kernel's device time, not the host's
+    launch latency."""
     import torch
 
     import pose_retrieved_kv_b200 as P
@@ -249,10 +282,16 @@ def run_kernel_only(args, local_rank: int):
     lay = P.make_layout(**cfg)
     _, lblk, _, T = P.prsink_layout_tokens(lay)
     H, d = cfg["n_heads"], cfg["head_dim"]
-    nbuf = 2
-    q = [synth.normal_bf16((lblk, H, d), 5 + i, 0).to(dev) for i in range(nbuf)]
-    k = [synth.normal_bf16((H, T, d), 5 + i, 1).to(dev) for i in range(nbuf)]
-    v = [synth.normal_bf16((H, T, d), 5 + i, 2).to(dev) for i in range(nbuf)]
+    if args.only == "attention":
+        nbuf = 2                                 # 2 x (q + k + v) = 2 x 322 MB at 480x480
+        q = [synth.normal_bf16((lblk, H, d), 5 + i, 0).to(dev) for i in range(nbuf)]
+        k = [synth.normal_bf16((H, T, d), 5 + i, 1).to(dev) for i in range(nbuf)]
+        v = [synth.normal_bf16((H, T, d), 5 + i, 2).to(dev) for i in range(nbuf)]
+    else:
+        nbuf = 6                                 # 6 block sources (166 MB at 480x480)
+        q = [synth.normal_bf16((lblk, H, d), 5 + i, 0).to(dev) for i in range(nbuf)]
+        k = [torch.zeros((H, T, d), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+        v = [torch.zeros((H, T, d), dtype=torch.bfloat16, device=dev) for _ in range(2)]
     out = torch.empty((lblk, H, d), dtype=torch.bfloat16, device=dev)
 
     def launch(i):
@@ -260,12 +299,15 @@ def run_kernel_only(args, local_rank: int):
         if args.only == "attention":
             P.prsink_attention(lay, q[j], k[j], v[j], out)
         else:
-            P.prsink_kv_append(lay, q[j], q[(j + 1) % nbuf], k[j], v[j], P.SLOT_RING0)
+            # ring slot (i mod 3) of one of two caches: consecutive launches write 55 MB apart
+            P.prsink_kv_append(lay, q[j], q[(j + 3) % nbuf], k[i % 2], v[i % 2],
+                               P.SLOT_RING0 + (i // 2) % 3)
 
     for i in range(args.warmup):
         launch(i)
     torch.cuda.synchronize()
     times = []
+    torch.cuda._sleep(int(2e6 + 4e5 * args.steps))    # ~1 ms + ~0.2 ms per launch at 2 GHz
     for i in range(args.steps):
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
@@ -291,6 +333,9 @@ def run_kernel_only(args, local_rank: int):
         roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm"],
                 "unit": "GB/s", "frac": round(ach / peaks["hbm"], 4),
                 "peak_source": f"{peaks['source']} hbm_gbs"}
+    src, prof = (ATTN_SRC, ATTN_PROFILE) if args.only == "attention" else (APPEND_SRC, APPEND_PROFILE)
+    roof["traffic"] = _profiled_traffic(src, prof) if args.config == "480x480" else None
+    roof["traffic_source"] = f"{prof}: ncu dram bytes read + written per launch"
     return {"kernel": args.only, "config": args.config, "avg_ms": round(avg, 4),
             "min_ms": round(min(ms), 4), "max_ms": round(max(ms), 4), "launches": len(ms),
             "roofline": roof}
