@@ -44,6 +44,34 @@ append_kernel(const uint4* __restrict__ k_new, const uint4* __restrict__ v_new,
   }
 }
 
+// Row-tiled form for C = 8 or 16 chunks per row (head_dim 64 or 128): block (x, h, kv) moves
+// tokens [x*R*U, (x+1)*R*U) of head h, R = 256/C rows per pass, U passes with all loads issued
+// before the stores.  No integer division: the chunk and row of a thread are a mask and a shift.
+template <int C, int U>
+__global__ void __launch_bounds__(kCopyThreads)
+append_rows_kernel(const uint4* __restrict__ k_new, const uint4* __restrict__ v_new,
+                   uint4* __restrict__ k_cache, uint4* __restrict__ v_cache, uint32_t n,
+                   uint32_t H, uint64_t T, uint64_t start) {
+  constexpr int R = kCopyThreads / C;
+  const uint4* __restrict__ src = blockIdx.z ? v_new : k_new;
+  uint4* __restrict__ dst = blockIdx.z ? v_cache : k_cache;
+  const uint32_t h = blockIdx.y;
+  const uint32_t c = threadIdx.x & (C - 1);
+  const uint32_t tok0 = blockIdx.x * (R * U) + threadIdx.x / C;
+  uint4 v[U];
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    const uint32_t tok = tok0 + u * R;
+    if (tok < n) v[u] = __ldcs(src + (static_cast<uint64_t>(tok) * H + h) * C + c);
+  }
+  uint4* __restrict__ row = dst + (static_cast<uint64_t>(h) * T + start) * C + c;
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    const uint32_t tok = tok0 + u * R;
+    if (tok < n) row[static_cast<uint64_t>(tok) * C] = v[u];
+  }
+}
+
 // Segment copy: segment y (one (layer, k|v, head) run of `seg_chunks` contiguous chunks) from
 // src + y-dependent offset to dst + y-dependent offset.  Runs only if *flag != 0 (flag may be
 // null) and *sel >= 0; *sel picks the bank entry on the bank side.
@@ -175,12 +203,29 @@ extern "C" int prsink_kv_append(const prsink_layout* layout, const void* k_new,
   const uint32_t C = layout->head_dim * 2 / 16;
   const uint64_t chunks = n * layout->n_heads * C;
   if (chunks == 0) return PRSINK_OK;
-  dim3 grid(grid_for(chunks), 2);
-  append_kernel<<<grid, kCopyThreads, 0, static_cast<cudaStream_t>(stream)>>>(
-      static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new),
-      static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache),
-      static_cast<uint32_t>(chunks), layout->n_heads, C, static_cast<uint64_t>(g.T),
-      static_cast<uint64_t>(g.slot_start[dest_slot]));
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const auto* kn = static_cast<const uint4*>(k_new);
+  const auto* vn = static_cast<const uint4*>(v_new);
+  auto* kc = static_cast<uint4*>(k_cache);
+  auto* vc = static_cast<uint4*>(v_cache);
+  const uint64_t start = static_cast<uint64_t>(g.slot_start[dest_slot]);
+  constexpr int kU = 4;
+  if (C == 16 || C == 8) {
+    const uint32_t rows_per_block = (kCopyThreads / C) * kU;
+    dim3 grid(static_cast<unsigned>((n + rows_per_block - 1) / rows_per_block),
+              static_cast<unsigned>(layout->n_heads), 2);
+    if (C == 16)
+      append_rows_kernel<16, kU><<<grid, kCopyThreads, 0, st>>>(
+          kn, vn, kc, vc, static_cast<uint32_t>(n), layout->n_heads, g.T, start);
+    else
+      append_rows_kernel<8, kU><<<grid, kCopyThreads, 0, st>>>(
+          kn, vn, kc, vc, static_cast<uint32_t>(n), layout->n_heads, g.T, start);
+  } else {
+    dim3 grid(grid_for(chunks), 2);
+    append_kernel<<<grid, kCopyThreads, 0, st>>>(kn, vn, kc, vc, static_cast<uint32_t>(chunks),
+                                                 layout->n_heads, C, static_cast<uint64_t>(g.T),
+                                                 start);
+  }
   count_launch();
   return check_launch("prsink_kv_append");
 }

@@ -18,10 +18,23 @@ def _bits(t: torch.Tensor) -> np.ndarray:
     return t.detach().cpu().view(torch.int16).numpy()
 
 
-@pytest.mark.parametrize("name", ["tiny", "480x480", "384x672_r4"])
+# head_dim 32 (4 chunks per row) takes the generic chunk-indexed kernel, 64 and 128 the
+# row-tiled one; the odd grids leave ragged last token blocks
+APPEND_EXTRA = {
+    "d32_5x7": dict(n_heads=3, head_dim=32, grid_h=5, grid_w=7, frames_per_block=3, ref_frames=1,
+                    ring_slots=3, rope_mode=3, rope_split=(12, 10, 10), rope_base=10000.0),
+    "d64_9x5": dict(n_heads=2, head_dim=64, grid_h=9, grid_w=5, frames_per_block=2, ref_frames=1,
+                    ring_slots=2, rope_mode=3, rope_split=(24, 20, 20), rope_base=10000.0),
+}
+
+
+@pytest.mark.parametrize("name", ["tiny", "480x480", "384x672_r4", "d32_5x7", "d64_9x5"])
 def test_kv_append_bit_exact_all_slots(name):
     need_gpu()
-    cfg = synth.preset(name, block_index=5, valid_mask=0xFF)
+    if name in APPEND_EXTRA:
+        cfg = dict(APPEND_EXTRA[name], block_index=5, valid_mask=0xFF)
+    else:
+        cfg = synth.preset(name, block_index=5, valid_mask=0xFF)
     s = oracle.layout_sizes(cfg)
     H, d, T = cfg["n_heads"], cfg["head_dim"], s["T"]
     lay = P.make_layout(**cfg)
