@@ -52,11 +52,15 @@ def _peaks():
 
 def _profiled_traffic(src_rel: str, profile_rel: str):
     """DRAM bytes per launch (read + write) recorded from an ncu capture in ``profiles/``, or
-    None when the kernel source has changed since that capture (sha256 mismatch)."""
+    None when the kernel's sources (its .cu file and the shared device header) have changed
+    since that capture (sha256 mismatch)."""
     import hashlib
     try:
-        with open(os.path.join(ROOT, src_rel), "rb") as f:
-            digest = hashlib.sha256(f.read()).hexdigest()
+        h = hashlib.sha256()
+        for rel in (src_rel, KERNEL_HEADER):
+            with open(os.path.join(ROOT, rel), "rb") as f:
+                h.update(f.read())
+        digest = h.hexdigest()
         with open(os.path.join(ROOT, profile_rel)) as f:
             text = f.read()
     except OSError:
@@ -70,6 +74,7 @@ def _profiled_traffic(src_rel: str, profile_rel: str):
     return rec_bytes if rec_hash == digest else None
 
 
+KERNEL_HEADER = "pose_retrieved_kv_b200/csrc/prsink_internal.cuh"
 ATTN_SRC = "pose_retrieved_kv_b200/csrc/attention_sm100.cu"
 ATTN_PROFILE = "profiles/attention_480x480.md"
 APPEND_SRC = "pose_retrieved_kv_b200/csrc/kv_copy.cu"
