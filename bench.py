@@ -39,6 +39,25 @@ M_BANK = 5
 WRITE_BLOCKS = 20
 
 
+def max_over_ranks(x: float, device, world: int) -> float:
+    """Max of a per-rank timing over all ranks (the job takes as long as its slowest rank); the
+    identity on one rank.  `device` is where the reduction tensor lives (cuda for NCCL, cpu for
+    gloo)."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(n_layers: int, steps: int, world: int, seconds: float) -> float:
+    """Layer-blocks per second of the whole job: every rank runs `steps` blocks of `n_layers`
+    layers on its own replica, and the job's time is the slowest rank's."""
+    return n_layers * steps * world / seconds
+
+
 def _peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -220,10 +239,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     if P.prsink_sync_status() != P.PRSINK_OK:
         raise RuntimeError("device status reported a timeout in the timed region")
     attn_ms = [a.elapsed_time(b) for a, b in attn_events]
-    if world > 1:
-        tt = torch.tensor([ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = max_over_ranks(ms, dev, world)
 
     e2e = None
     if not args.no_e2e:
@@ -232,8 +248,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     if rank != 0:
         return None
     peaks = _peaks()
-    layer_blocks = n_layers * args.steps * world
-    value = layer_blocks / (ms / 1e3)
+    value = job_throughput(n_layers, args.steps, world, ms / 1e3)
     flops = 4.0 * lblk * T * d * H                      # QK^T + PV, steady state: all keys valid
     attn_avg_ms = statistics.mean(attn_ms)
     achieved = flops / (attn_avg_ms / 1e3) / 1e12
@@ -424,14 +439,10 @@ def run_e2e(args, st, qkv, kp_all, ok_all, dev, world):
     for k in range(args.steps):
         block(first + 2 + k)
     torch.cuda.synchronize()
-    el = time.perf_counter() - t0
-    if world > 1:
-        tt = torch.tensor([el], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        el = float(tt.item())
+    el = max_over_ranks(time.perf_counter() - t0, dev, world)
     if P.prsink_sync_status() != P.PRSINK_OK:
         raise RuntimeError("device status reported a timeout in the e2e run")
-    return {"value": round(n_layers * args.steps * world / el, 3), "unit": UNIT,
+    return {"value": round(job_throughput(n_layers, args.steps, world, el), 3), "unit": UNIT,
             "h2d_bytes_per_step": bytes_in // args.steps,
             "d2h_bytes_per_step": bytes_out // args.steps}
 
