@@ -86,7 +86,7 @@ def _profiled_traffic(src_rel: str, profile_rel: str):
         return None
     rec_hash = rec_bytes = None
     for line in text.splitlines():
-        if line.startswith("kernel source sha256:"):
+        if line.startswith("kernel source sha256"):
             rec_hash = line.split(":", 1)[1].strip()
         elif line.startswith("DRAM bytes per launch (read + write):"):
             rec_bytes = int(line.split(":", 1)[1].strip())
@@ -302,7 +302,26 @@ def run_kernel_only(args, local_rank: int):
     lay = P.make_layout(**cfg)
     _, lblk, _, T = P.prsink_layout_tokens(lay)
     H, d = cfg["n_heads"], cfg["head_dim"]
-    if args.only == "attention":
+    fill_layers = 8
+    if args.only == "dynfill":
+        # bank of M entries x 8 layers and an 8-layer cache (~4.6 GB at 480x480); the query
+        # fingerprint alternates between two bank entries, so every call moves the retrieved
+        # entry's K/V into the dynamic slot of all 8 layers (0.88 GB read + 0.88 GB written)
+        g = torch.Generator().manual_seed(11)
+        bank_phi = torch.nn.functional.normalize(
+            torch.randn(M_BANK, P.FP_DIM, generator=g, dtype=torch.float64), dim=1).float().to(dev)
+        bank_src = torch.arange(M_BANK, dtype=torch.int64, device=dev)
+        bank_count = torch.tensor([M_BANK], dtype=torch.int32, device=dev)
+        r_out = torch.zeros(1, dtype=torch.int32, device=dev)
+        score_out = torch.zeros(1, dtype=torch.float32, device=dev)
+        copy_out = torch.zeros(1, dtype=torch.int32, device=dev)
+        dyn_src = torch.full((1,), -1, dtype=torch.int64, device=dev)
+        bank_kv = torch.empty((fill_layers, M_BANK, 2, H, lblk, d), dtype=torch.bfloat16, device=dev)
+        bank_kv.view(-1)[::4099] = 1.0
+        cache_kv = torch.zeros((fill_layers, 2, H, T, d), dtype=torch.bfloat16, device=dev)
+        nbuf = 2
+        q = k = v = None
+    elif args.only == "attention":
         nbuf = 2                                 # 2 x (q + k + v) = 2 x 322 MB at 480x480
         q = [synth.normal_bf16((lblk, H, d), 5 + i, 0).to(dev) for i in range(nbuf)]
         k = [synth.normal_bf16((H, T, d), 5 + i, 1).to(dev) for i in range(nbuf)]
@@ -312,11 +331,15 @@ def run_kernel_only(args, local_rank: int):
         q = [synth.normal_bf16((lblk, H, d), 5 + i, 0).to(dev) for i in range(nbuf)]
         k = [torch.zeros((H, T, d), dtype=torch.bfloat16, device=dev) for _ in range(2)]
         v = [torch.zeros((H, T, d), dtype=torch.bfloat16, device=dev) for _ in range(2)]
-    out = torch.empty((lblk, H, d), dtype=torch.bfloat16, device=dev)
+    out = torch.empty((lblk, H, d), dtype=torch.bfloat16, device=dev) if q is not None else None
 
     def launch(i):
         j = i % nbuf
-        if args.only == "attention":
+        if args.only == "dynfill":
+            P.prsink_retrieve(lay, bank_phi[j], bank_phi, bank_src, bank_count, M_BANK, -10,
+                              r_out, score_out, copy_out, dyn_src, bank_kv, cache_kv,
+                              fill_layers)
+        elif args.only == "attention":
             P.prsink_attention(lay, q[j], k[j], v[j], out)
         else:
             # ring slot (i mod 3) of one of two caches: consecutive launches write 55 MB apart
@@ -348,14 +371,22 @@ def run_kernel_only(args, local_rank: int):
                 "unit": "TFLOP/s", "frac": round(ach / peaks["bf16"], 4),
                 "peak_source": f"{peaks['source']} bf16_tflops (burst)"}
     else:
-        work = 2.0 * 2 * lblk * H * d * 2                   # K and V: read + write
+        # append: K and V of one block, read + written; dynamic fill: K and V of one bank entry
+        # for every layer, read + written (the retrieval kernel's 11 KB are not counted)
+        work = 2.0 * 2 * lblk * H * d * 2 * (fill_layers if args.only == "dynfill" else 1)
         ach = work / (avg / 1e3) / 1e9
         roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm"],
                 "unit": "GB/s", "frac": round(ach / peaks["hbm"], 4),
                 "peak_source": f"{peaks['source']} hbm_gbs"}
-    src, prof = (ATTN_SRC, ATTN_PROFILE) if args.only == "attention" else (APPEND_SRC, APPEND_PROFILE)
-    roof["traffic"] = _profiled_traffic(src, prof) if args.config == "480x480" else None
-    roof["traffic_source"] = f"{prof}: ncu dram bytes read + written per launch"
+    if args.only == "dynfill":
+        roof["traffic"] = None
+        if int(copy_out.item()) != 1:
+            raise RuntimeError("the dynamic fill did not copy on the last call")
+    else:
+        src, prof = ((ATTN_SRC, ATTN_PROFILE) if args.only == "attention"
+                     else (APPEND_SRC, APPEND_PROFILE))
+        roof["traffic"] = _profiled_traffic(src, prof) if args.config == "480x480" else None
+        roof["traffic_source"] = f"{prof}: ncu dram bytes read + written per launch"
     return {"kernel": args.only, "config": args.config, "avg_ms": round(avg, 4),
             "min_ms": round(min(ms), 4), "max_ms": round(max(ms), 4), "launches": len(ms),
             "roofline": roof}
@@ -540,7 +571,7 @@ def main():
                     help="heads of the CPU oracle sample in the cpu_baseline leg (~10-30 s)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["attention", "append"], default=None,
+    ap.add_argument("--only", choices=["attention", "append", "dynfill"], default=None,
                     help="time one kernel alone at the workload's sizes (for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
