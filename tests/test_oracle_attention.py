@@ -7,7 +7,9 @@
 * special cases: zero queries average the valid values, one valid key returns its value,
   no valid key returns zeros;
 * the attention is unchanged when every slot is moved to another physical place as long as the
-  logical layout is kept (ring rotation with the block index).
+  logical layout is kept (ring rotation with the block index);
+* on the tiny layout the float64 oracle agrees with an independent long-double computation to
+  1e-12 (its own rounding, nothing more).
 """
 import cmath
 import math
@@ -231,3 +233,50 @@ def test_position_probe_catches_one_misplaced_key(monkeypatch):
         bad, _ = oracle.attention(cfg, q, k, v, rows=rows)
         monkeypatch.setattr(po, "key_positions", orig)
         assert np.abs(bad - good).max() > 0.25, name
+
+
+def _longdouble_attention(cfg, q, k, v):
+    """The tiny 1-D layout in numpy long double (80-bit on x86-64): gather the logical sequence,
+    rotate every pair by its position's angle, textbook softmax.  Independent of the oracle's
+    code; it bounds the oracle's float64 rounding."""
+    ld = np.longdouble
+    lf, lblk, _ = _sizes(cfg)
+    d = cfg["head_dim"]
+    rows = _logical_rows(cfg)
+    n_log = len(rows)
+    j = np.arange(d // 2, dtype=ld)
+    inv = np.power(ld(cfg["rope_base"]), -2 * j / ld(d))
+
+    def rot(x, pos):
+        ang = np.asarray(pos, dtype=ld)[:, None] * inv[None, :]
+        c, s = np.cos(ang), np.sin(ang)
+        x0, x1 = x[:, 0::2], x[:, 1::2]
+        out = np.empty_like(x)
+        out[:, 0::2] = x0 * c - x1 * s
+        out[:, 1::2] = x0 * s + x1 * c
+        return out
+
+    valid = [(r, i) for i, (r, ok) in enumerate(rows) if ok]
+    phys = [r for r, _ in valid]
+    logi = [i for _, i in valid]
+    out = np.zeros((lblk, cfg["n_heads"], d), dtype=ld)
+    for h in range(cfg["n_heads"]):
+        kk = rot(k[h][phys].astype(ld), logi)
+        vv = v[h][phys].astype(ld)
+        qq = rot(q[:, h].astype(ld), [n_log - lblk + i for i in range(lblk)])
+        sc = (qq @ kk.T) / np.sqrt(ld(d))
+        sc -= sc.max(axis=1, keepdims=True)
+        w = np.exp(sc)
+        out[:, h] = (w @ vv) / w.sum(axis=1, keepdims=True)
+    return out
+
+
+@pytest.mark.skipif(np.finfo(np.longdouble).eps >= np.finfo(np.float64).eps,
+                    reason="long double is not wider than double on this platform")
+@pytest.mark.parametrize("b,mask", [(7, 0b111111), (2, 0b011011)])
+def test_float64_oracle_within_rounding_of_long_double(b, mask):
+    cfg = synth.preset("tiny", block_index=b, valid_mask=mask)
+    q, k, v = _inputs(cfg, 21 + b)
+    got, _ = oracle.attention(cfg, q, k, v)
+    ref = _longdouble_attention(cfg, q, k, v)
+    assert np.abs(got - ref.astype(np.float64)).max() < 1e-12
