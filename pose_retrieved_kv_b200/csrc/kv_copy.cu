@@ -162,8 +162,10 @@ int launch_bank_cache_copy(const prsink_layout* L, const Geometry& g, int M, int
     set_error("too many (layer, k/v, head) segments: %llu", (unsigned long long)segs);
     return PRSINK_ERR_ARG;
   }
-  // enough CTAs in flight for HBM: about 4 per SM over all segments
-  uint64_t gx = (148ull * 4 + segs - 1) / segs;
+  // about 32 CTAs per SM over all segments (four waves of eight resident 256-thread CTAs), so
+  // that the last wave is a small share of the copy: with one CTA per segment, 640 segments
+  // (8 layers) sat unevenly on 148 SMs (4 or 5 each) and reached 0.73 of the copy peak
+  uint64_t gx = (148ull * 32 + segs - 1) / segs;
   const uint64_t gmax = (bank_head + kCopyThreads * kCopyUnroll - 1) / (kCopyThreads * kCopyUnroll);
   if (gx > gmax) gx = gmax;
   if (gx < 1) gx = 1;
