@@ -4,7 +4,7 @@ Argument marshalling only: every function checks the torch tensors it is given (
 contiguity, size), passes their data pointers and the current CUDA stream to the C entry point
 of the same name, and raises :class:`PRSinkError` on a non-zero status.  All computation happens
 in the library's CUDA kernels; there is no fallback of any kind.  If the library has not been
-built (``python -m pose_retrieved_kv_b200.build``) importing this module raises.
+built (``python pose_retrieved_kv_b200/build.py``) importing this module raises.
 """
 from __future__ import annotations
 
@@ -69,7 +69,7 @@ def make_layout(n_heads, head_dim, grid_h, grid_w, frames_per_block=3, ref_frame
 def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"{LIB_PATH} is missing: build it with "
-                          "`python -m pose_retrieved_kv_b200.build` (needs nvcc)")
+                          "`python pose_retrieved_kv_b200/build.py` (needs nvcc)")
     lib = ctypes.CDLL(LIB_PATH)
     vp, ll, i, f = ctypes.c_void_p, ctypes.c_longlong, ctypes.c_int, ctypes.c_float
     lp = ctypes.POINTER(Layout)

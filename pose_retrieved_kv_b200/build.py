@@ -1,6 +1,7 @@
 """Build ``libprsink.so`` in-tree with nvcc for sm_100a.
 
-Usage: ``python -m pose_retrieved_kv_b200.build [-v]``.  The library is self-contained (static
+Usage: ``python pose_retrieved_kv_b200/build.py [-v]`` (run as a script: importing the package
+loads the library, which does not exist yet on a fresh checkout).  The library is self-contained (static
 CUDA runtime, driver entry points looked up at run time), so it loads next to PyTorch's own
 runtime without extra linking.
 """

@@ -4,6 +4,7 @@ import ctypes
 import os
 import re
 import subprocess
+import sys
 
 import pytest
 
@@ -96,3 +97,13 @@ def test_rope_table_limit_reported():
     lay = P.make_layout(**{**synth.preset("480x480"), "rope_mode": 1, "rope_split": (128, 0, 0)})
     assert _lib().prsink_attention(ctypes.byref(lay), 16, 16, 16, 16, None, None,
                                    None) == P.PRSINK_ERR_UNSUPPORTED
+
+
+def test_build_module_loads_without_the_package():
+    """build() must work on a fresh checkout, where the library does not exist yet: loading
+    the build script may not import the package (whose import loads the library)."""
+    code = ("import sys, __graft_entry__ as g; m = g._build_module(); "
+            "assert callable(m.build) and m.ARCH; "
+            "assert 'pose_retrieved_kv_b200' not in sys.modules, 'package imported'")
+    res = subprocess.run([sys.executable, "-c", code], cwd=ROOT, capture_output=True, text=True)
+    assert res.returncode == 0, res.stderr
