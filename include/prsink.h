@@ -18,7 +18,10 @@
  *   - Return value: PRSINK_OK (0) or a negative PRSINK_ERR_* code.  Invalid arguments are
  *     rejected on the host before anything is launched.  No C++ exception crosses the ABI.
  *   - Device-side waits are bounded.  A wait that runs out records PRSINK_ERR_TIMEOUT in a
- *     device status word; prsink_sync_status() reads and clears it.
+ *     device status word; prsink_sync_status() reads and clears it.  There is ONE status word
+ *     per device, shared by every stream and host thread that uses the library on it: a
+ *     timeout raised by a kernel on stream A is reported (and cleared) by a
+ *     prsink_sync_status() call made for stream B.
  *
  * Cache layout (the "slot-indexed" cache).  For one layer, K and V caches are each
  * bf16 [H][T][d] (head-major, d contiguous).  Physical key rows are grouped in slots:
@@ -154,6 +157,10 @@ int prsink_fingerprint(const float* kp, const unsigned char* frame_ok, float* ph
  *               On return it is bank_src[r] (or -1 when r = -1).
  *   bank_kv, cache_kv, n_layers: optional (all NULL/0 to skip the copy).  When given, the
  *               dynamic slot of every layer is overwritten with bank entry r iff *copy_out.
+ *               The copy addresses bank_kv as bf16 [n_layers][M][2][H][L_blk][d] and cache_kv
+ *               as bf16 [n_layers][2][H][T][d] (H, d, L_blk, T from `layout`): the caller must
+ *               pass buffers of exactly these sizes (the library cannot check device sizes;
+ *               the Python binding does).
  * Similarities are accumulated in float64.  Errors: PRSINK_ERR_ARG, _ALIGN, _LAUNCH. */
 int prsink_retrieve(const prsink_layout* layout, const float* phi_b, const float* bank_phi,
                     const long long* bank_src, const int* bank_count, int M,
@@ -176,15 +183,18 @@ int prsink_retrieve(const prsink_layout* layout, const float* phi_b, const float
  *   action_out int32 scalar (written): slot written, or -1
  *   cache_kv, bank_kv, n_layers: optional (NULL/0 to skip).  When given and action >= 0, the
  *               clean K/V of block b (ring slot b mod R of every layer) is copied into bank
- *               entry `action`.
+ *               entry `action`.  Sizes as for prsink_retrieve: bank_kv bf16
+ *               [n_layers][M][2][H][L_blk][d], cache_kv bf16 [n_layers][2][H][T][d].
  * Errors: PRSINK_ERR_ARG, PRSINK_ERR_ALIGN, PRSINK_ERR_LAUNCH. */
 int prsink_bank_update(const prsink_layout* layout, float* bank_phi, long long* bank_src,
                        int* bank_count, int M, const float* phi_b, long long b,
                        int write_blocks, int* action_out, const void* cache_kv, void* bank_kv,
                        int n_layers, void* stream);
 
-/* Synchronise `stream`, then read and clear the device status word: PRSINK_OK, or
- * PRSINK_ERR_TIMEOUT if a bounded wait ran out since the last call, or PRSINK_ERR_LAUNCH. */
+/* Synchronise `stream`, then read and clear the status word of the current device:
+ * PRSINK_OK, or PRSINK_ERR_TIMEOUT if a bounded wait of any kernel on this device (any
+ * stream) ran out since the word was last cleared, or PRSINK_ERR_LAUNCH.  Only `stream` is
+ * synchronised: kernels still running on other streams may report later. */
 int prsink_sync_status(void* stream);
 
 /* Text of the last host-side error of this thread ("" if none).  Owned by the library. */

@@ -120,15 +120,34 @@ def _ptr(t: Optional[torch.Tensor], name: str, dtype=None, numel=None, device=Tr
         return 0
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
-    if device and not t.is_cuda:
-        raise ValueError(f"{name} must be a CUDA tensor")
     if dtype is not None and t.dtype != dtype:
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     if numel is not None and t.numel() != numel:
         raise ValueError(f"{name} must hold {numel} elements, got {t.numel()}")
+    if device and not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
     return t.data_ptr()
+
+
+def _kv_sizes(layout: Optional[Layout], M: int, n_layers: int, bank_kv, cache_kv):
+    """Element counts the copy kernels address: bank_kv [n_layers][M][2][H][L_blk][d] and
+    cache_kv [n_layers][2][H][T][d] (None, None when no copy is requested)."""
+    if bank_kv is None and cache_kv is None and not n_layers:
+        return None, None
+    if layout is None:
+        raise ValueError("the K/V copy needs a layout")
+    _, lblk, _, T = prsink_layout_tokens(layout)
+    H, d = layout.n_heads, layout.head_dim
+    n_bank, n_cache = n_layers * M * 2 * H * lblk * d, n_layers * 2 * H * T * d
+    # checked before any other argument: a wrong size here would make a copy kernel run past
+    # the end of a buffer
+    for t, name, n in ((bank_kv, "bank_kv", n_bank), (cache_kv, "cache_kv", n_cache)):
+        if isinstance(t, torch.Tensor) and t.numel() != n:
+            raise ValueError(f"{name} must hold {n} elements for this layout, M = {M} and "
+                             f"n_layers = {n_layers}, got {t.numel()}")
+    return n_bank, n_cache
 
 
 def prsink_version() -> int:
@@ -187,6 +206,7 @@ def prsink_fingerprint(kp, frame_ok, phi, stream=None):
 def prsink_retrieve(layout: Optional[Layout], phi_b, bank_phi, bank_src, bank_count, M: int,
                     exclude_block: int, r_out, score_out, copy_out, dyn_src, bank_kv=None,
                     cache_kv=None, n_layers: int = 0, stream=None):
+    n_bank, n_cache = _kv_sizes(layout, M, n_layers, bank_kv, cache_kv)
     rc = _lib.prsink_retrieve(
         ctypes.byref(layout) if layout is not None else None,
         _ptr(phi_b, "phi_b", torch.float32, FP_DIM),
@@ -195,22 +215,23 @@ def prsink_retrieve(layout: Optional[Layout], phi_b, bank_phi, bank_src, bank_co
         int(M), int(exclude_block), _ptr(r_out, "r_out", torch.int32, 1),
         _ptr(score_out, "score_out", torch.float32, 1),
         _ptr(copy_out, "copy_out", torch.int32, 1), _ptr(dyn_src, "dyn_src", torch.int64, 1),
-        _ptr(bank_kv, "bank_kv", torch.bfloat16), _ptr(cache_kv, "cache_kv", torch.bfloat16),
-        int(n_layers), _stream(stream))
+        _ptr(bank_kv, "bank_kv", torch.bfloat16, n_bank),
+        _ptr(cache_kv, "cache_kv", torch.bfloat16, n_cache), int(n_layers), _stream(stream))
     _check(rc, "prsink_retrieve")
 
 
 def prsink_bank_update(layout: Optional[Layout], bank_phi, bank_src, bank_count, M: int, phi_b,
                        b: int, write_blocks: int, action_out, cache_kv=None, bank_kv=None,
                        n_layers: int = 0, stream=None):
+    n_bank, n_cache = _kv_sizes(layout, M, n_layers, bank_kv, cache_kv)
     rc = _lib.prsink_bank_update(
         ctypes.byref(layout) if layout is not None else None,
         _ptr(bank_phi, "bank_phi", torch.float32, M * FP_DIM),
         _ptr(bank_src, "bank_src", torch.int64, M), _ptr(bank_count, "bank_count", torch.int32, 1),
         int(M), _ptr(phi_b, "phi_b", torch.float32, FP_DIM), int(b), int(write_blocks),
         _ptr(action_out, "action_out", torch.int32, 1),
-        _ptr(cache_kv, "cache_kv", torch.bfloat16), _ptr(bank_kv, "bank_kv", torch.bfloat16),
-        int(n_layers), _stream(stream))
+        _ptr(cache_kv, "cache_kv", torch.bfloat16, n_cache),
+        _ptr(bank_kv, "bank_kv", torch.bfloat16, n_bank), int(n_layers), _stream(stream))
     _check(rc, "prsink_bank_update")
 
 

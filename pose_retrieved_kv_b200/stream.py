@@ -35,7 +35,13 @@ def stream_valid_mask(ring_slots: int, b: int) -> int:
 
 
 class PRSinkStream:
-    """Caches, bank and decisions of one stream for ``n_layers`` attention layers."""
+    """Caches, bank and decisions of one stream for ``n_layers`` attention layers.
+
+    Nothing here synchronises, so a bounded device wait that ran out (the attention kernel
+    then writes zeros for the affected rows and records a timeout in the device status word)
+    is not noticed by these calls: check once per block, with ``end_block(check=True)`` or
+    ``check_status()``, which synchronise the stream and raise ``PRSinkError`` on a timeout.
+    """
 
     def __init__(self, cfg: dict, n_layers: int, M: int = 5, write_blocks: int = 20,
                  device="cuda"):
@@ -90,9 +96,20 @@ class PRSinkStream:
             L.prsink_kv_append(lay, k_new, v_new, k, v, L.SLOT_STATIC, stream)
         L.prsink_attention(lay, q, k, v, out, lse, self.dyn_src, stream)
 
-    def end_block(self, stream=None):
-        """Bank update with the clean K/V of block b, then advance to block b+1."""
+    def end_block(self, stream=None, check: bool = False):
+        """Bank update with the clean K/V of block b, then advance to block b+1.  With
+        ``check`` the stream is synchronised and a device timeout raises."""
         L.prsink_bank_update(self.layout(), self.bank_phi, self.bank_src, self.bank_count,
                              self.M, self.phi, self.b, self.write_blocks, self.action,
                              self.cache_kv, self.bank_kv, self.n_layers, stream)
         self.b += 1
+        if check:
+            self.check_status(stream)
+
+    @staticmethod
+    def check_status(stream=None):
+        """Synchronise ``stream`` and raise ``PRSinkError`` if a bounded device wait ran out
+        (on any stream of this device) since the status word was last read."""
+        rc = L.prsink_sync_status(stream)
+        if rc != L.PRSINK_OK:
+            raise L.PRSinkError(rc, "PRSinkStream", L.prsink_last_error())

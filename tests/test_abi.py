@@ -107,3 +107,37 @@ def test_build_module_loads_without_the_package():
             "assert 'pose_retrieved_kv_b200' not in sys.modules, 'package imported'")
     res = subprocess.run([sys.executable, "-c", code], cwd=ROOT, capture_output=True, text=True)
     assert res.returncode == 0, res.stderr
+
+
+def test_copy_buffers_sized_for_the_layout_or_rejected_before_launch():
+    """The dynamic fill and the bank store address bank_kv and cache_kv from the layout, M and
+    n_layers alone: the binding checks both sizes on the host before anything is launched."""
+    import torch
+    cfg = synth.preset("tiny")
+    lay = P.make_layout(**cfg)
+    _, lblk, _, T = P.prsink_layout_tokens(lay)
+    M, n_layers = 5, 2
+    f32 = lambda n: torch.zeros(n, dtype=torch.float32)       # noqa: E731
+    i32 = lambda n: torch.zeros(n, dtype=torch.int32)         # noqa: E731
+    i64 = lambda n: torch.zeros(n, dtype=torch.int64)         # noqa: E731
+    bf = lambda n: torch.zeros(n, dtype=torch.bfloat16)       # noqa: E731
+    good_bank, good_cache = n_layers * M * 2 * lblk * 64, n_layers * 2 * T * 64
+    before = P.prsink_launch_count()
+    for bank_n, cache_n, what in [(good_bank - 64, good_cache, "bank_kv"),
+                                  (good_bank, good_cache + 64, "cache_kv"),
+                                  (n_layers * 4 * 2 * lblk * 64, good_cache, "bank_kv")]:
+        with pytest.raises(ValueError, match=what):
+            P.prsink_retrieve(lay, f32(558), f32(M * 558), i64(M), i32(1), M, 0, i32(1),
+                              None, i32(1), i64(1), bf(bank_n), bf(cache_n), n_layers)
+        with pytest.raises(ValueError, match=what):
+            P.prsink_bank_update(lay, f32(M * 558), i64(M), i32(1), M, f32(558), 0, 20,
+                                 i32(1), bf(cache_n), bf(bank_n), n_layers)
+    # a wrong n_layers for the given buffers
+    with pytest.raises(ValueError, match="bank_kv"):
+        P.prsink_retrieve(lay, f32(558), f32(M * 558), i64(M), i32(1), M, 0, i32(1), None,
+                          i32(1), i64(1), bf(good_bank), bf(good_cache), n_layers + 1)
+    # right sizes on host tensors: rejected for the device, not for the size
+    with pytest.raises(ValueError, match="CUDA"):
+        P.prsink_retrieve(lay, f32(558), f32(M * 558), i64(M), i32(1), M, 0, i32(1), None,
+                          i32(1), i64(1), bf(good_bank), bf(good_cache), n_layers)
+    assert P.prsink_launch_count() == before

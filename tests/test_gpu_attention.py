@@ -2,7 +2,8 @@
 
 Tiny layouts are compared element by element over every query; the full workload sizes
 (480x480, 384x672 with 3 and 4 ring slots, 672x384) run in the same launch configuration as the
-benchmark and are compared on sampled query rows of every head, including the ragged last tile.
+benchmark and are compared on sampled query rows of every head, including the ragged last tile,
+and on every row of a few heads.
 """
 import numpy as np
 import pytest
@@ -11,8 +12,12 @@ import torch
 import oracle
 import pose_retrieved_kv_b200 as P
 import synth
-from tests._gpu import (LSE_MAX_ABS, attention_inputs, check_attention, f64, need_gpu)
+from tests._gpu import (ATTN_MAX_ABS, ATTN_MEAN_ABS, LSE_MAX_ABS, attention_inputs,
+                        check_attention, f64, need_gpu)
+from tests._cases import (GAIN_CASES, RESCALE_CASES, gain_case, rescale_case,
+                          sample_rows)
 from tests._probe import probe_inputs
+from tests._rounding import model_errors, rescaled_rows
 
 pytestmark = pytest.mark.gpu
 
@@ -65,54 +70,68 @@ def test_small_3d_every_element(ci, b, mask):
     assert np.abs(lse - ref_lse).max() <= LSE_MAX_ABS
 
 
+# Inputs whose logits reach far beyond those of N(0,1) draws exceed the stated tolerance
+# through the bf16 rounding of the rotated q and k alone (tests/_rounding.py; pinned on the CPU
+# in tests/test_rounding_model.py): there the bound is 1.5 x the rounding model's error on the
+# same inputs, and the stated tolerance where that is larger.
+MODEL_FACTOR = 1.5
+
+
+def _model_bounds(cfg, q, k, v, rows, ref, ref_lse):
+    emax, emean, else_ = model_errors(cfg, f64(q), f64(k), f64(v), rows, ref, ref_lse)
+    return (max(ATTN_MAX_ABS, MODEL_FACTOR * emax), max(ATTN_MEAN_ABS, MODEL_FACTOR * emean),
+            max(LSE_MAX_ABS, MODEL_FACTOR * else_))
+
+
 @pytest.mark.parametrize("S,sign", [(5.0, -1.0), (60.0, -1.0), (900.0, -1.0), (60.0, 1.0),
                                     (900.0, 1.0)])
 def test_scores_far_from_zero(S, sign):
     """Every score about sign * S (tests/_probe.py): the running max must follow rows whose
     scores are all large negative or large positive (a max stuck at 0 underflows every weight
-    and returns LSE = -inf, O = 0).  The kernel rounds rotated q and k to bf16, so score errors
-    grow like 2^-9 * |score|: the bounds scale with S."""
+    and returns LSE = -inf, O = 0)."""
     need_gpu()
     cfg = synth.preset("tiny", block_index=7, valid_mask=0xFF)
     q, k, v = probe_inputs(cfg, S, seed=3, sign=sign)
     got, lse = _run(cfg, q, k, v)
+    rows = np.arange(48)
     ref, ref_lse = oracle.attention(cfg, f64(q), f64(k), f64(v))
+    bmax, bmean, blse = _model_bounds(cfg, q, k, v, rows, ref, ref_lse)
     assert np.all(np.isfinite(lse))
-    assert np.abs(lse - ref_lse).max() <= 2e-2 + 2.5e-3 * S
-    assert np.abs(got - ref).max() <= 2e-2 + 1e-4 * S
+    assert np.abs(lse - ref_lse).max() <= blse
+    err = np.abs(got - ref)
+    assert err.max() <= bmax and err.mean() <= bmean, (err.max(), err.mean(), bmax, bmean)
     assert np.abs(got).max() > 0.1 * np.abs(ref).max()        # not an all-zero output
 
 
-@pytest.mark.parametrize("name,slot,gain", [("tiny", 5, 6.0), ("480x480", 5, 5.0),
-                                            ("480x480", 0, 5.0)])
+@pytest.mark.parametrize("name,slot,gain", GAIN_CASES)
 def test_max_growing_or_shrinking_across_tiles(name, slot, gain):
-    """Keys of one slot scaled by `gain`: when it is the last slot the row max grows by far
-    more than 2^8 between key tiles, so the output accumulator is rescaled mid-row; when it
-    is the ref slot (first tiles) later tiles sit far below the max instead."""
+    """Keys of one slot scaled by `gain` (logits up to ~24): when it is the last slot the row
+    max grows by far more than 2^8 between key tiles, so the output accumulator is rescaled
+    mid-row; when it is the ref slot (first tiles) later tiles sit far below the max."""
     need_gpu()
-    cfg = synth.preset(name, block_index=1000, valid_mask=0xFF)
-    if name != "tiny":
-        cfg = dict(cfg, n_heads=4)
-    q, k, v = attention_inputs(cfg, seed=13)
-    a, e = oracle.slot_ranges(cfg)[slot]
-    k = k.clone()
-    k[:, a:e] = (k[:, a:e].float() * gain).to(torch.bfloat16)
+    cfg, q, k, v, rows = gain_case(name, slot, gain)
     got, lse = _run(cfg, q, k, v)
-    s = oracle.layout_sizes(cfg)
-    rows = _sample_rows(s["L_blk"], 9) if name != "tiny" else np.arange(s["L_blk"])
     ref, ref_lse = oracle.attention(cfg, f64(q), f64(k), f64(v), rows=rows)
-    # bf16 rounding of the rotated q and k moves a logit by ~2^-9 |logit|; with logits up to
-    # s_max (>> the ~4 of N(0,1) inputs) the softmax is sharp, so the bound grows with s_max
-    kpos, _ = oracle.key_positions(cfg)
-    qpos = oracle.query_positions(cfg)
-    s_max = max(np.abs(oracle.rope_rotate(cfg, f64(q)[rows, h], qpos[rows])
-                       @ oracle.rope_rotate(cfg, f64(k)[h], kpos).T).max()
-                for h in range(cfg["n_heads"])) / np.sqrt(cfg["head_dim"])
-    bound = 2e-2 * max(1.0, s_max / 8.0)
+    bmax, bmean, blse = _model_bounds(cfg, q, k, v, rows, ref, ref_lse)
     err = np.abs(got[rows] - ref)
-    assert np.all(np.isfinite(got)) and err.max() <= bound, (err.max(), bound)
-    assert err.mean() <= 2e-3 * max(1.0, s_max / 8.0)
-    assert np.abs(lse[:, rows] - ref_lse).max() <= LSE_MAX_ABS * max(1.0, s_max / 8.0)
+    assert np.all(np.isfinite(got))
+    assert err.max() <= bmax and err.mean() <= bmean, (err.max(), err.mean(), bmax, bmean)
+    assert np.abs(lse[:, rows] - ref_lse).max() <= blse
+
+
+@pytest.mark.parametrize("name,gain", RESCALE_CASES)
+def test_rescale_path_at_stated_tolerance(name, gain):
+    """Logits below ~10 whose row max still jumps by more than 2^8 between key tiles on a good
+    share of rows (counted on the CPU from the oracle's scores in the kernel's tile order): the
+    accumulator rescale is exercised under the stated tolerance itself."""
+    need_gpu()
+    cfg, q, k, v, rows = rescale_case(name, gain)
+    assert np.mean(np.concatenate([rescaled_rows(cfg, f64(q), f64(k), rows, h)
+                                   for h in range(cfg["n_heads"])])) >= 0.15
+    got, lse = _run(cfg, q, k, v)
+    ref, ref_lse = oracle.attention(cfg, f64(q), f64(k), f64(v), rows=rows)
+    check_attention(got[rows], ref, f"rescale {name}")
+    assert np.abs(lse[:, rows] - ref_lse).max() <= LSE_MAX_ABS
 
 
 def test_no_valid_key_gives_zeros():
@@ -150,12 +169,6 @@ def test_empty_slots_holding_nan_are_ignored():
     check_attention(got, ref, "nan in empty slot")
 
 
-def _sample_rows(lblk, seed):
-    g = np.random.default_rng(seed)
-    edge = [0, 1, 127, 128, lblk - 13, lblk - 12, lblk - 1]
-    return np.unique(np.concatenate([edge, g.choice(lblk, 40, replace=False)]))
-
-
 @pytest.mark.parametrize("name", ["480x480", "384x672", "384x672_r4", "672x384"])
 def test_full_size_sampled_rows(name):
     need_gpu()
@@ -163,11 +176,25 @@ def test_full_size_sampled_rows(name):
     q, k, v = attention_inputs(cfg, seed=2)
     got, lse = _run(cfg, q, k, v)
     s = oracle.layout_sizes(cfg)
-    rows = _sample_rows(s["L_blk"], 7)
+    rows = sample_rows(s["L_blk"], 7)
     ref, ref_lse = oracle.attention(cfg, f64(q), f64(k), f64(v), rows=rows)
     check_attention(got[rows], ref, name)
     assert np.abs(lse[:, rows] - ref_lse).max() <= LSE_MAX_ABS
     assert np.all(np.isfinite(got))
+
+
+@pytest.mark.parametrize("name,heads", [("480x480", [0, 13, 26, 39]),
+                                        ("384x672_r4", [0, 39])])
+def test_full_size_every_row_of_some_heads(name, heads):
+    """Every query row (every query tile, the ragged last one included) of a few heads at the
+    full workload size, in the launch configuration the benchmark times (all 40 heads)."""
+    need_gpu()
+    cfg = synth.preset(name, block_index=1000, valid_mask=0xFF)
+    q, k, v = attention_inputs(cfg, seed=2)
+    got, lse = _run(cfg, q, k, v)
+    ref, ref_lse = oracle.attention(cfg, f64(q), f64(k), f64(v), heads=heads)
+    check_attention(got[:, heads], ref, f"{name} all rows")
+    assert np.abs(lse[heads] - ref_lse).max() <= LSE_MAX_ABS
 
 
 def test_full_size_early_block():
@@ -176,7 +203,7 @@ def test_full_size_early_block():
     cfg = synth.preset("480x480", block_index=1, valid_mask=0b0011011)
     q, k, v = attention_inputs(cfg, seed=6)
     got, _ = _run(cfg, q, k, v)
-    rows = _sample_rows(2700, 8)
+    rows = sample_rows(2700, 8)
     ref, _ = oracle.attention(cfg, f64(q), f64(k), f64(v), rows=rows, heads=[0, 17, 39])
     check_attention(got[rows][:, [0, 17, 39]], ref, "480x480 b=1")
 
