@@ -7,13 +7,23 @@ attention over ref 900 + static 2700 + dynamic 2700 + 3 x 2700 ring = 14400 keys
 update.  The bank (M = 5) is filled during the first 20 blocks, which run untimed before the
 warm-up; the timed blocks are the steady state after it is frozen.
 
-Metric: blocks/s per 40-head layer (layer-blocks per second over all GPUs), with the attention
-TFLOP/s and its fraction of the measured dense bf16 peak.  Inputs are synthetic (N(0,1) bf16
-Q/K/V, clustered synthetic poses); per-layer caches are 295 MB and 40 layers are cycled, so
-every launch reads from HBM (the working set is far above the 126 MB L2).
+Metric: blocks/s per 40-head layer (layer-blocks per second of the whole job), with the
+attention TFLOP/s and its fraction of the measured dense bf16 peak.  Inputs are synthetic
+(N(0,1) bf16 Q/K/V, clustered synthetic poses); per-layer caches are 295 MB and 40 layers are
+cycled, so every launch reads from HBM (the working set is far above the 126 MB L2).
+
+At one GPU the line also carries sub-records: each kernel timed alone (KV append, the 40-layer
+dynamic-sink fill, attention at the 3024-query layouts, attention on rotating and on repeated
+inputs) and a 300-block stream from block 0 (bank written during the first 20 blocks, then
+frozen), end to end on the device.
+
+``--gpus N`` runs one process per GPU (started here through torch.distributed.run when no
+launcher did).  ``--partition heads`` (default) splits the 40 heads of every cache and bank
+entry over the ranks, as the pages' Ulysses layout does, with the pose decisions replicated:
+one stream, strong scaling.  ``--partition replicas`` runs an independent stream per rank
+(weak scaling).  No collective is on the data path either way.
 
 ``--impl reference`` times the float64 CPU oracle on a bounded sample of the same workload.
-Under torchrun every rank runs its own stream (weak scaling, no data-path collective).
 """
 from __future__ import annotations
 
@@ -52,10 +62,11 @@ def max_over_ranks(x: float, device, world: int) -> float:
     return float(t.item())
 
 
-def job_throughput(n_layers: int, steps: int, world: int, seconds: float) -> float:
-    """Layer-blocks per second of the whole job: every rank runs `steps` blocks of `n_layers`
-    layers on its own replica, and the job's time is the slowest rank's."""
-    return n_layers * steps * world / seconds
+def job_throughput(n_layers: int, steps: int, streams: int, seconds: float) -> float:
+    """Layer-blocks per second of the whole job: each of `streams` independent streams (one per
+    rank for replicas, one for the whole job when the heads are split) runs `steps` blocks of
+    `n_layers` layers, and the job's time is the slowest rank's."""
+    return n_layers * steps * streams / seconds
 
 
 def _peaks():
@@ -157,8 +168,233 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------------------------------
+# kernels timed alone
+# ------------------------------------------------------------------------------------------
+
+def time_launches(launch, warmup: int, steps: int):
+    """Per-launch device times (ms) of ``launch(i)``: ``warmup`` untimed launches, then
+    ``steps`` launches each between two CUDA events on the current stream.  A device-side sleep
+    is queued ahead of the timed launches so that the host has enqueued them all before the
+    first one starts: each event pair then brackets one kernel's device time, not the host's
+    launch latency."""
+    import torch
+    for i in range(warmup):
+        launch(i)
+    torch.cuda.synchronize()
+    ev = []
+    torch.cuda._sleep(int(2e6 + 4e5 * steps))        # ~1 ms + ~0.2 ms per launch at 2 GHz
+    for i in range(steps):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        launch(warmup + i)
+        e1.record()
+        ev.append((e0, e1))
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in ev]
+
+
+def _summary(ms, work, unit, peak, peak_source):
+    avg = statistics.mean(ms)
+    scale = 1e12 if unit == "TFLOP/s" else 1e9
+    ach = work / (avg / 1e3) / scale
+    return {"avg_ms": round(avg, 4), "min_ms": round(min(ms), 4), "max_ms": round(max(ms), 4),
+            "launches": len(ms), "achieved": round(ach, 1), "unit": unit, "peak": peak,
+            "frac": round(ach / peak, 4), "peak_source": peak_source}
+
+
+def attention_alone(name: str, warmup: int, steps: int, repeat: bool = False, nbuf: int = 2):
+    """One attention call at a workload's full size (block 1000, every slot valid), timed
+    alone.  ``repeat`` = the same inputs every launch; otherwise ``nbuf`` input sets (each
+    larger than L2) alternate."""
+    import torch
+
+    import pose_retrieved_kv_b200 as P
+    import synth
+
+    cfg = synth.preset(name, block_index=1000, valid_mask=0xFF)
+    lay = P.make_layout(**cfg)
+    _, lblk, _, T = P.prsink_layout_tokens(lay)
+    H, d = cfg["n_heads"], cfg["head_dim"]
+    n = 1 if repeat else nbuf
+    q = [synth.normal_bf16((lblk, H, d), 5 + i, 0).cuda() for i in range(n)]
+    k = [synth.normal_bf16((H, T, d), 5 + i, 1).cuda() for i in range(n)]
+    v = [synth.normal_bf16((H, T, d), 5 + i, 2).cuda() for i in range(n)]
+    out = torch.empty((lblk, H, d), dtype=torch.bfloat16, device="cuda")
+    ms = time_launches(lambda i: P.prsink_attention(lay, q[i % n], k[i % n], v[i % n], out),
+                       warmup, steps)
+    if P.prsink_sync_status() != P.PRSINK_OK:
+        raise RuntimeError("device status reported a timeout")
+    peaks = _peaks()
+    rec = _summary(ms, 4.0 * lblk * T * d * H, "TFLOP/s", peaks["bf16"],
+                   f"{peaks['source']} bf16_tflops (burst)")
+    rec.update(queries=lblk, keys=T, gflop=round(4.0 * lblk * T * d * H / 1e9, 1),
+               inputs="repeated" if repeat else f"{n} sets of {(lblk + 2 * T) * H * d * 2 / 1e6:.0f} MB alternating")
+    return rec
+
+
+def append_alone(name: str, warmup: int, steps: int):
+    """prsink_kv_append of one block into a ring slot, timed alone: six source blocks and two
+    caches rotate, so consecutive launches touch different memory."""
+    import torch
+
+    import pose_retrieved_kv_b200 as P
+    import synth
+
+    cfg = synth.preset(name, block_index=1000, valid_mask=0xFF)
+    lay = P.make_layout(**cfg)
+    _, lblk, _, T = P.prsink_layout_tokens(lay)
+    H, d = cfg["n_heads"], cfg["head_dim"]
+    nbuf = 6
+    src = [synth.normal_bf16((lblk, H, d), 5 + i, 0).cuda() for i in range(nbuf)]
+    k = [torch.zeros((H, T, d), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+    v = [torch.zeros((H, T, d), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+
+    def launch(i):
+        j = i % nbuf
+        P.prsink_kv_append(lay, src[j], src[(j + 3) % nbuf], k[i % 2], v[i % 2],
+                           P.SLOT_RING0 + (i // 2) % 3)
+
+    ms = time_launches(launch, warmup, steps)
+    peaks = _peaks()
+    work = 2.0 * 2 * lblk * H * d * 2          # K and V, read + written
+    rec = _summary(ms, work, "GB/s", peaks["hbm"], f"{peaks['source']} hbm_gbs")
+    rec.update(bytes_per_launch=int(work), inputs=f"{nbuf} source blocks x 2 caches rotating")
+    return rec
+
+
+def dynfill_alone(st, warmup: int, steps: int):
+    """The dynamic-sink fill of every layer of a stream (prsink_retrieve with the copy), timed
+    alone on the stream's own 40-layer cache and bank: the query fingerprint alternates between
+    two bank entries, so every call moves a different entry's K/V of all layers."""
+    import torch
+
+    import pose_retrieved_kv_b200 as P
+
+    lay = st.layout()
+    count = int(st.bank_count.item())
+    if count < 2:
+        return None
+    phis = [st.bank_phi[j].clone() for j in range(2)]
+    r = torch.zeros(1, dtype=torch.int32, device=st.bank_phi.device)
+    sc = torch.zeros(1, dtype=torch.float32, device=st.bank_phi.device)
+    cp = torch.zeros(1, dtype=torch.int32, device=st.bank_phi.device)
+    dyn = torch.full((1,), -1, dtype=torch.int64, device=st.bank_phi.device)
+
+    def launch(i):
+        P.prsink_retrieve(lay, phis[i % 2], st.bank_phi, st.bank_src, st.bank_count, st.M,
+                          -10, r, sc, cp, dyn, st.bank_kv, st.cache_kv, st.n_layers)
+
+    ms = time_launches(launch, warmup, steps)
+    if int(cp.item()) != 1:
+        raise RuntimeError("the dynamic fill did not copy on the last call")
+    peaks = _peaks()
+    work = 2.0 * 2 * st.L_blk * st.cfg["n_heads"] * st.cfg["head_dim"] * 2 * st.n_layers
+    rec = _summary(ms, work, "GB/s", peaks["hbm"], f"{peaks['source']} hbm_gbs")
+    rec.update(layers=st.n_layers, bytes_per_call=int(work),
+               note="one call = the retrieval kernel + the predicated copy of every layer")
+    return rec
+
+
+def kernel_records(st, args):
+    """Sub-records of the one-GPU line: every kernel the benchmark spec's targets name, timed alone."""
+    w, k = 3, 20
+    rec = {"append_480x480": append_alone("480x480", w, 50),
+           "dynfill_40_layers": dynfill_alone(st, w, 10),
+           "attention_480x480_rotating": attention_alone("480x480", w, k),
+           "attention_480x480_repeat": attention_alone("480x480", w, k, repeat=True)}
+    for name in ("384x672", "384x672_r4", "672x384"):
+        rec[f"attention_{name}"] = attention_alone(name, w, k)
+    rec["note"] = ("attention: burst bf16 peak (a kernel timed alone); 'rotating' alternates "
+                   "two input sets of 322 MB, 'repeat' reuses one (K/V of 295 MB exceed the "
+                   "126 MB L2 either way)")
+    return rec
+
+
+# ------------------------------------------------------------------------------------------
 # our arm
 # ------------------------------------------------------------------------------------------
+
+def _inputs(args, cfg_full, rank, world, dev):
+    """Per-pass Q/K/V pool, ref K/V per layer and poses of this rank.  With the head partition
+    every rank draws the whole job's inputs (same seeds) and keeps its heads; replicas draw
+    their own."""
+    import synth
+    from pose_retrieved_kv_b200 import shard
+
+    split = args.partition == "heads" and world > 1
+    seed0 = 0 if split else 1000 * rank
+    H, d = cfg_full["n_heads"], cfg_full["head_dim"]
+    lf = cfg_full["grid_h"] * cfg_full["grid_w"]
+    lblk, lref = lf * cfg_full["frames_per_block"], lf * cfg_full["ref_frames"]
+
+    def mine(x):
+        return shard.shard_tokens(x, world, rank) if split else x
+
+    qkv = [[mine(synth.normal_bf16((lblk, H, d), 100 + seed0 + i, j)).to(dev) for j in range(3)]
+           for i in range(args.pool)]
+    ref = [mine(synth.normal_bf16((lref, H, d), 7 + seed0 + layer, 1)).to(dev)
+           for layer in range(args.layers)]
+    return qkv, ref, 11 + (0 if split else rank)
+
+
+def _block(st, P, b, kp_dev, ok_dev, qkv, out, events=None, stream=None):
+    """One block of the stream: retrieval + dynamic fill, per layer 3 denoising passes and the
+    Clean KV Update pass (append + attention), bank update."""
+    import torch
+    st.begin_block(kp_dev[b], ok_dev[b])
+    i = 0
+    pool = len(qkv)
+    for layer in range(st.n_layers):
+        for p in range(PASSES):
+            q, kn, vn = qkv[(b * st.n_layers * PASSES + i) % pool]
+            i += 1
+            lay = st.layout()
+            k, v = st.kv(layer)
+            P.prsink_kv_append(lay, kn, vn, k, v, P.SLOT_RING0 + st.b % st.R)
+            if p == PASSES - 1 and st.b == 0:
+                P.prsink_kv_append(lay, kn, vn, k, v, P.SLOT_STATIC)
+            if events is not None:
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+            P.prsink_attention(lay, q, k, v, out, None, st.dyn_src)
+            if events is not None:
+                e1.record(stream)
+                events.append((e0, e1))
+    st.end_block()
+
+
+def run_stream(st, P, kp_dev, ok_dev, qkv, out, n_blocks, dev):
+    """A whole stream from block 0 (bank written during the first blocks, then frozen),
+    timed on the device with the inputs resident; counts the dynamic fills and bank writes on
+    the device."""
+    import torch
+    st.reset()
+    fills = torch.zeros(1, dtype=torch.int32, device=dev)
+    writes = torch.zeros(1, dtype=torch.int32, device=dev)
+    n0 = P.prsink_launch_count()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for b in range(n_blocks):
+        _block(st, P, b, kp_dev, ok_dev, qkv, out)
+        fills += st.copied
+        writes += (st.action >= 0).to(torch.int32)
+    t1.record()
+    torch.cuda.synchronize()
+    if P.prsink_sync_status() != P.PRSINK_OK:
+        raise RuntimeError("device status reported a timeout in the stream")
+    s = t0.elapsed_time(t1) / 1e3
+    return {"blocks": n_blocks, "layers": st.n_layers, "seconds": round(s, 3),
+            "blocks_per_s": round(n_blocks / s, 3),
+            "layer_blocks_per_s": round(n_blocks * st.n_layers / s, 3),
+            "dynamic_fills": int(fills.item()), "bank_writes": int(writes.item()),
+            "gpu_launches": int(P.prsink_launch_count() - n0),
+            "inputs": "resident in HBM; poses from 12 recurring clusters (sigma 0.03), 5 % "
+                      "failed frames; bank M = 5 written during the first 20 blocks"}
+
 
 def run_ours(args, rank: int, world: int, local_rank: int):
     import torch
@@ -166,54 +402,49 @@ def run_ours(args, rank: int, world: int, local_rank: int):
 
     import pose_retrieved_kv_b200 as P
     import synth
+    from pose_retrieved_kv_b200 import shard
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    cfg = synth.preset(args.config)
+    stream_only = args.config == "stream300"
+    cfg_full = synth.preset("480x480" if stream_only else args.config)
+    split = args.partition == "heads" and world > 1
+    cfg = shard.shard_config(cfg_full, world, rank) if split else cfg_full
     n_layers = args.layers
     H, d = cfg["n_heads"], cfg["head_dim"]
     st = P.PRSinkStream(cfg, n_layers=n_layers, M=M_BANK, write_blocks=WRITE_BLOCKS, device=dev)
     lblk, T = st.L_blk, st.T
-    # a pool of distinct per-pass inputs (well above L2), reused round-robin over layer-passes
-    pool = args.pool
-    qkv = [[synth.normal_bf16((lblk, H, d), 100 + rank * 1000 + i, j).to(dev) for j in range(3)]
-           for i in range(pool)]
+    qkv, ref, pose_seed = _inputs(args, cfg_full, rank, world, dev)
     for layer in range(n_layers):
-        kr = synth.normal_bf16((st.L_ref, H, d), 7 + layer, 1).to(dev)
-        st.set_ref(layer, kr, kr)
-    n_blocks = WRITE_BLOCKS + args.warmup + args.steps
-    kp_all, ok_all, _ = synth.pose_stream(11 + rank, n_blocks)
+        st.set_ref(layer, ref[layer], ref[layer])
+    n_blocks = max(WRITE_BLOCKS + args.warmup + args.steps + 2, args.stream_blocks)
+    kp_all, ok_all, _ = synth.pose_stream(pose_seed, n_blocks)
     kp_dev = torch.from_numpy(np.ascontiguousarray(kp_all[:, :, :62, :])).to(dev)
     ok_dev = torch.from_numpy(ok_all).to(dev)
     out = torch.empty((lblk, H, d), dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream(dev)
+    streams = 1 if split else world             # independent streams in the job
+
+    if stream_only:
+        if world > 1:
+            dist.barrier()
+        rec = run_stream(st, P, kp_dev, ok_dev, qkv, out, args.stream_blocks, dev)
+        s = max_over_ranks(rec["seconds"], dev, world)
+        if rank != 0:
+            return None
+        return {"metric": METRIC, "value": round(n_layers * args.stream_blocks * streams / s, 3),
+                "unit": UNIT, "n_gpus": world, "steps": args.stream_blocks, "warmup": 0,
+                "ms_per_step": round(1e3 * s / args.stream_blocks, 3), "higher_is_better": True,
+                "scaling": "strong" if split else "weak", "vs_baseline": None, "dtype": "bf16",
+                "data": "synthetic", "gpu_launches": rec["gpu_launches"],
+                "config": {"workload": f"{args.stream_blocks}-block stream at 480x480 from "
+                                       "block 0, 40 layers x 4 passes per block",
+                           "parallelism": _parallelism(args, world)},
+                "stream": rec}
 
     attn_events = []
-
-    def block(b, timed):
-        st.begin_block(kp_dev[b], ok_dev[b])
-        i = 0
-        for layer in range(n_layers):
-            for p in range(PASSES):
-                q, kn, vn = qkv[(b * n_layers * PASSES + i) % pool]
-                i += 1
-                lay = st.layout()
-                k, v = st.kv(layer)
-                P.prsink_kv_append(lay, kn, vn, k, v, P.SLOT_RING0 + st.b % st.R)
-                if p == PASSES - 1 and st.b == 0:
-                    P.prsink_kv_append(lay, kn, vn, k, v, P.SLOT_STATIC)
-                if timed:
-                    e0 = torch.cuda.Event(enable_timing=True)
-                    e1 = torch.cuda.Event(enable_timing=True)
-                    e0.record(stream)
-                P.prsink_attention(lay, q, k, v, out, None, st.dyn_src)
-                if timed:
-                    e1.record(stream)
-                    attn_events.append((e0, e1))
-        st.end_block()
-
     for b in range(WRITE_BLOCKS + args.warmup):          # bank fill + warm-up, untimed
-        block(b, False)
+        _block(st, P, b, kp_dev, ok_dev, qkv, out)
     torch.cuda.synchronize()
     if P.prsink_sync_status() != P.PRSINK_OK:
         raise RuntimeError("device status reported a timeout during warm-up")
@@ -228,7 +459,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record(stream)
     for k in range(args.steps):
-        block(WRITE_BLOCKS + args.warmup + k, True)
+        _block(st, P, WRITE_BLOCKS + args.warmup + k, kp_dev, ok_dev, qkv, out, attn_events,
+               stream)
     t1.record(stream)
     torch.cuda.synchronize()
     if world > 1:
@@ -243,12 +475,16 @@ def run_ours(args, rank: int, world: int, local_rank: int):
 
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(args, st, qkv, kp_all, ok_all, dev, world)
+        e2e = run_e2e(args, st, qkv, kp_all, ok_all, dev, world, streams)
+    extras = stream_rec = None
+    if world == 1 and not args.no_extras:
+        extras = kernel_records(st, args)
+        stream_rec = run_stream(st, P, kp_dev, ok_dev, qkv, out, args.stream_blocks, dev)
 
     if rank != 0:
         return None
     peaks = _peaks()
-    value = job_throughput(n_layers, args.steps, world, ms / 1e3)
+    value = job_throughput(n_layers, args.steps, streams, ms / 1e3)
     flops = 4.0 * lblk * T * d * H                      # QK^T + PV, steady state: all keys valid
     attn_avg_ms = statistics.mean(attn_ms)
     achieved = flops / (attn_avg_ms / 1e3) / 1e12
@@ -256,22 +492,24 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     res = {
         "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 3),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "strong" if split else "weak",
+        "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (N(0,1) bf16 Q/K/V, clustered synthetic poses; no weights needed)",
         "config": {"workload": f"per-block step {args.config}: {n_layers} layers x "
                                f"({PASSES - 1} denoise + 1 clean) x (append + PR-Sink attention), "
                                "retrieval + dynamic fill, bank update",
-                   "heads": H, "head_dim": d, "queries": lblk, "keys": T,
-                   "ring_slots": cfg["ring_slots"], "layers": n_layers, "bank": M_BANK,
+                   "heads": cfg_full["n_heads"], "heads_per_gpu": H, "head_dim": d,
+                   "queries": lblk, "keys": T, "ring_slots": cfg["ring_slots"],
+                   "layers": n_layers, "bank": M_BANK,
                    "l2": "inputs larger than L2 (295 MB cache per layer, layers cycled)",
-                   "parallelism": f"replica x{world} (independent streams)"},
+                   "parallelism": _parallelism(args, world)},
         "attention": {"avg_ms": round(attn_avg_ms, 4), "tflops": round(achieved, 1),
                       "frac_of_bf16_peak": round(achieved / peak, 4),
-                      "launches_timed": len(attn_ms)},
+                      "launches_timed": len(attn_ms), "rank": 0},
         "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
                      "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
                      "traffic": (_profiled_traffic(ATTN_SRC, ATTN_PROFILE)
-                                 if args.config == "480x480" else None),
+                                 if args.config == "480x480" and H == 40 else None),
                      "traffic_source": f"{ATTN_PROFILE}: ncu dram__bytes_read.sum + "
                                        "dram__bytes_write.sum, bytes per launch",
                      "peak_source": f"{peaks['source']} bf16_tflops_sustained"},
@@ -280,122 +518,59 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     }
     if e2e is not None:
         res["e2e"] = e2e
+    if extras is not None:
+        res["kernels"] = extras
+    if stream_rec is not None:
+        res["stream300"] = stream_rec
     if not args.no_cpu_baseline and world == 1:
         res["cpu_baseline"] = cpu_baseline(args, cfg)
     return res
 
 
+def _parallelism(args, world):
+    if world == 1:
+        return "single GPU"
+    if args.partition == "heads":
+        return f"heads split over {world} GPUs (one stream; pose decisions replicated)"
+    return f"replica x{world} (independent streams)"
+
+
 def run_kernel_only(args, local_rank: int):
-    """Time one kernel alone (``--only attention|append``) at the workload's sizes: W warm-up
-    launches, then K launches on rotating buffers (a set larger than L2).  A device-side sleep
-    is queued ahead of the timed launches so that the host has enqueued them all before the
-    first one starts: each event pair then brackets one kernel's device time, not the host's
-    launch latency."""
+    """Time one kernel alone (``--only attention|append|dynfill``) at the workload's sizes
+    (for profiling: one process, few launches)."""
     import torch
 
     import pose_retrieved_kv_b200 as P
     import synth
 
     torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
-    cfg = synth.preset(args.config, block_index=1000, valid_mask=0xFF)
-    lay = P.make_layout(**cfg)
-    _, lblk, _, T = P.prsink_layout_tokens(lay)
-    H, d = cfg["n_heads"], cfg["head_dim"]
-    fill_layers = 8
-    if args.only == "dynfill":
-        # bank of M entries x 8 layers and an 8-layer cache (~4.6 GB at 480x480); the query
-        # fingerprint alternates between two bank entries, so every call moves the retrieved
-        # entry's K/V into the dynamic slot of all 8 layers (0.88 GB read + 0.88 GB written)
-        g = torch.Generator().manual_seed(11)
-        bank_phi = torch.nn.functional.normalize(
-            torch.randn(M_BANK, P.FP_DIM, generator=g, dtype=torch.float64), dim=1).float().to(dev)
-        bank_src = torch.arange(M_BANK, dtype=torch.int64, device=dev)
-        bank_count = torch.tensor([M_BANK], dtype=torch.int32, device=dev)
-        r_out = torch.zeros(1, dtype=torch.int32, device=dev)
-        score_out = torch.zeros(1, dtype=torch.float32, device=dev)
-        copy_out = torch.zeros(1, dtype=torch.int32, device=dev)
-        dyn_src = torch.full((1,), -1, dtype=torch.int64, device=dev)
-        bank_kv = torch.empty((fill_layers, M_BANK, 2, H, lblk, d), dtype=torch.bfloat16, device=dev)
-        bank_kv.view(-1)[::4099] = 1.0
-        cache_kv = torch.zeros((fill_layers, 2, H, T, d), dtype=torch.bfloat16, device=dev)
-        nbuf = 2
-        q = k = v = None
-    elif args.only == "attention":
-        nbuf = 2                                 # 2 x (q + k + v) = 2 x 322 MB at 480x480
-        q = [synth.normal_bf16((lblk, H, d), 5 + i, 0).to(dev) for i in range(nbuf)]
-        k = [synth.normal_bf16((H, T, d), 5 + i, 1).to(dev) for i in range(nbuf)]
-        v = [synth.normal_bf16((H, T, d), 5 + i, 2).to(dev) for i in range(nbuf)]
-    else:
-        nbuf = 6                                 # 6 block sources (166 MB at 480x480)
-        q = [synth.normal_bf16((lblk, H, d), 5 + i, 0).to(dev) for i in range(nbuf)]
-        k = [torch.zeros((H, T, d), dtype=torch.bfloat16, device=dev) for _ in range(2)]
-        v = [torch.zeros((H, T, d), dtype=torch.bfloat16, device=dev) for _ in range(2)]
-    out = torch.empty((lblk, H, d), dtype=torch.bfloat16, device=dev) if q is not None else None
-
-    def launch(i):
-        j = i % nbuf
-        if args.only == "dynfill":
-            P.prsink_retrieve(lay, bank_phi[j], bank_phi, bank_src, bank_count, M_BANK, -10,
-                              r_out, score_out, copy_out, dyn_src, bank_kv, cache_kv,
-                              fill_layers)
-        elif args.only == "attention":
-            P.prsink_attention(lay, q[j], k[j], v[j], out)
-        else:
-            # ring slot (i mod 3) of one of two caches: consecutive launches write 55 MB apart
-            P.prsink_kv_append(lay, q[j], q[(j + 3) % nbuf], k[i % 2], v[i % 2],
-                               P.SLOT_RING0 + (i // 2) % 3)
-
-    for i in range(args.warmup):
-        launch(i)
-    torch.cuda.synchronize()
-    times = []
-    torch.cuda._sleep(int(2e6 + 4e5 * args.steps))    # ~1 ms + ~0.2 ms per launch at 2 GHz
-    for i in range(args.steps):
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record()
-        launch(args.warmup + i)
-        e1.record()
-        times.append((e0, e1))
-    torch.cuda.synchronize()
-    if P.prsink_sync_status() != P.PRSINK_OK:
-        raise RuntimeError("device status reported a timeout")
-    ms = [a.elapsed_time(b) for a, b in times]
-    peaks = _peaks()
-    avg = statistics.mean(ms)
     if args.only == "attention":
-        work = 4.0 * lblk * T * d * H
-        ach = work / (avg / 1e3) / 1e12
-        roof = {"bound": "tensor", "achieved": round(ach, 1), "peak": peaks["bf16"],
-                "unit": "TFLOP/s", "frac": round(ach / peaks["bf16"], 4),
-                "peak_source": f"{peaks['source']} bf16_tflops (burst)"}
+        rec = attention_alone(args.config, args.warmup, args.steps)
+        rec["traffic"] = (_profiled_traffic(ATTN_SRC, ATTN_PROFILE)
+                          if args.config == "480x480" else None)
+    elif args.only == "append":
+        rec = append_alone(args.config, args.warmup, args.steps)
+        rec["traffic"] = (_profiled_traffic(APPEND_SRC, APPEND_PROFILE)
+                          if args.config == "480x480" else None)
     else:
-        # append: K and V of one block, read + written; dynamic fill: K and V of one bank entry
-        # for every layer, read + written (the retrieval kernel's 11 KB are not counted)
-        work = 2.0 * 2 * lblk * H * d * 2 * (fill_layers if args.only == "dynfill" else 1)
-        ach = work / (avg / 1e3) / 1e9
-        roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm"],
-                "unit": "GB/s", "frac": round(ach / peaks["hbm"], 4),
-                "peak_source": f"{peaks['source']} hbm_gbs"}
-    if args.only == "dynfill":
-        roof["traffic"] = None
-        if int(copy_out.item()) != 1:
-            raise RuntimeError("the dynamic fill did not copy on the last call")
-    else:
-        src, prof = ((ATTN_SRC, ATTN_PROFILE) if args.only == "attention"
-                     else (APPEND_SRC, APPEND_PROFILE))
-        roof["traffic"] = _profiled_traffic(src, prof) if args.config == "480x480" else None
-        roof["traffic_source"] = f"{prof}: ncu dram bytes read + written per launch"
-    return {"kernel": args.only, "config": args.config, "avg_ms": round(avg, 4),
-            "min_ms": round(min(ms), 4), "max_ms": round(max(ms), 4), "launches": len(ms),
-            "roofline": roof}
+        cfg = synth.preset(args.config)
+        st = P.PRSinkStream(cfg, n_layers=args.layers, M=M_BANK, write_blocks=WRITE_BLOCKS,
+                            device=torch.device("cuda", local_rank))
+        g = torch.Generator().manual_seed(11)
+        st.bank_phi.copy_(torch.nn.functional.normalize(
+            torch.randn(M_BANK, P.FP_DIM, generator=g, dtype=torch.float64), dim=1).float())
+        st.bank_src.copy_(torch.arange(M_BANK))
+        st.bank_count.fill_(M_BANK)
+        st.bank_kv.view(-1)[::4099] = 1.0
+        rec = dynfill_alone(st, args.warmup, args.steps)
+    return {"kernel": args.only, "config": args.config, **rec}
 
 
-def run_e2e(args, st, qkv, kp_all, ok_all, dev, world):
+def run_e2e(args, st, qkv, kp_all, ok_all, dev, world, streams):
     """Same step through the public API with pinned HOST inputs and outputs: every step copies
     its poses and per-pass Q/K/V from the host and reads every attention output back.  Copies
-    run on their own streams, overlapped with compute through double buffering."""
+    run on their own streams, overlapped with compute through double buffering.  Timed with
+    CUDA events from the first copy to the last read-back, max over ranks."""
     import torch
     import torch.distributed as dist
 
@@ -466,14 +641,22 @@ def run_e2e(args, st, qkv, kp_all, ok_all, dev, world):
     if world > 1:
         dist.barrier()
     bytes_in = bytes_out = 0
-    t0 = time.perf_counter()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(comp)
+    h2d.wait_event(t0)
     for k in range(args.steps):
         block(first + 2 + k)
+    comp.wait_stream(h2d)
+    comp.wait_stream(d2h)
+    t1.record(comp)
     torch.cuda.synchronize()
-    el = max_over_ranks(time.perf_counter() - t0, dev, world)
+    if world > 1:
+        dist.barrier()
+    el = max_over_ranks(t0.elapsed_time(t1) / 1e3, dev, world)
     if P.prsink_sync_status() != P.PRSINK_OK:
         raise RuntimeError("device status reported a timeout in the e2e run")
-    return {"value": round(job_throughput(n_layers, args.steps, world, el), 3), "unit": UNIT,
+    return {"value": round(job_throughput(n_layers, args.steps, streams, el), 3), "unit": UNIT,
             "h2d_bytes_per_step": bytes_in // args.steps,
             "d2h_bytes_per_step": bytes_out // args.steps}
 
@@ -556,32 +739,60 @@ def run_reference(args, rank, world):
                     "d2h_bytes_per_step": 0}}
 
 
+def _launch_ranks(args) -> int:
+    """Start ``--gpus`` processes through torch.distributed.run (one per GPU, rendezvous on
+    127.0.0.1) running this script with the same arguments; returns their exit status."""
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           f"--nproc-per-node={args.gpus}", "--master-addr", "127.0.0.1",
+           "--master-port", str(port), os.path.abspath(__file__), *sys.argv[1:]]
+    return subprocess.call(cmd)
+
+
 def main():
-    ap = argparse.ArgumentParser(description=__doc__)
+    ap = argparse.ArgumentParser(description=__doc__,
+                                 formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", default="480x480")
+    ap.add_argument("--config", default="480x480",
+                    choices=["480x480", "384x672", "384x672_r4", "672x384", "stream300"])
+    ap.add_argument("--partition", choices=["heads", "replicas"], default="heads",
+                    help="N > 1: split the heads of one stream, or one stream per GPU")
     ap.add_argument("--layers", type=int, default=40)
     ap.add_argument("--pool", type=int, default=8)
+    ap.add_argument("--stream-blocks", type=int, default=300)
     ap.add_argument("--cpu-heads", type=int, default=4,
                     help="heads per step of the CPU oracle in --impl reference")
     ap.add_argument("--baseline-heads", type=int, default=40,
                     help="heads of the CPU oracle sample in the cpu_baseline leg (~10-30 s)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the kernel sub-records and the 300-block stream")
     ap.add_argument("--only", choices=["attention", "append", "dynfill"], default=None,
                     help="time one kernel alone at the workload's sizes (for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.gpus < 1:
+        ap.error("--gpus must be >= 1")
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        sys.exit(_launch_ranks(args))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if world != args.gpus:
-        world = max(world, 1)
+        sys.stderr.write(f"bench.py: --gpus {args.gpus} but the launcher started {world} "
+                         "ranks\n")
+        sys.exit(2)
     if args.only:
+        if world > 1:
+            ap.error("--only times one kernel on one GPU")
         res = run_kernel_only(args, local_rank)
     elif args.impl == "reference":
         res = run_reference(args, rank, world)

@@ -66,6 +66,16 @@ class PRSinkStream:
         self.action = torch.zeros(1, dtype=torch.int32, device=dev)
         self.b = 0
 
+    def reset(self):
+        """Start a new stream at block 0 on the same buffers: empty bank, empty dynamic sink.
+        The ref sink keeps its K/V; other slots are marked empty until written (their stale
+        bytes are never read)."""
+        self.bank_phi.zero_()
+        self.bank_src.fill_(-1)
+        self.bank_count.zero_()
+        self.dyn_src.fill_(-1)
+        self.b = 0
+
     def layout(self, b: int = None) -> L.Layout:
         b = self.b if b is None else b
         return L.make_layout(**{**self.cfg, "block_index": b,

@@ -68,3 +68,38 @@ def test_single_rank_is_identity():
     import bench
     assert bench.max_over_ranks(0.25, torch.device("cpu"), 1) == 0.25
     assert bench.job_throughput(40, 5, 1, 2.0) == pytest.approx(100.0)
+
+
+def test_gpus_mismatch_with_launcher_fails_loudly():
+    """A launcher that started fewer ranks than --gpus asks for must not time one GPU."""
+    env = dict(os.environ, WORLD_SIZE="1", RANK="0", LOCAL_RANK="0")
+    import subprocess
+    res = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2"],
+                         env=env, capture_output=True, text=True, timeout=120)
+    assert res.returncode == 2 and "--gpus 2" in res.stderr
+
+
+def test_gpus_without_launcher_starts_one_rank_per_gpu(monkeypatch):
+    """--gpus N with no launcher re-runs the script under torch.distributed.run with N ranks
+    on 127.0.0.1."""
+    sys.path.insert(0, ROOT)
+    import bench
+    seen = {}
+    monkeypatch.setattr(bench.subprocess, "call", lambda cmd: (seen.setdefault("cmd", cmd), 0)[1])
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--gpus", "4", "--steps", "2"])
+
+    class A:
+        gpus = 4
+    assert bench._launch_ranks(A()) == 0
+    cmd = seen["cmd"]
+    assert cmd[1:3] == ["-m", "torch.distributed.run"]
+    assert "--nproc-per-node=4" in cmd and "127.0.0.1" in cmd
+    assert cmd[-4:] == ["--gpus", "4", "--steps", "2"]
+
+
+def test_job_throughput_counts_streams_not_ranks_for_a_head_split():
+    sys.path.insert(0, ROOT)
+    import bench
+    # 4 ranks sharing one stream (heads split) vs 4 independent streams
+    assert bench.job_throughput(40, 5, 1, 2.0) == pytest.approx(100.0)
+    assert bench.job_throughput(40, 5, 4, 2.0) == pytest.approx(400.0)
