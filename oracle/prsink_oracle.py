@@ -31,6 +31,13 @@ What the oracle computes, function by function:
   bank_objective / bank_update diversity-driven replacement (mean pairwise similarity)
   valid_mask                   which slots hold data at block b
   stream_decisions             the per-block decision sequence of a stream
+  retrieve_fallback            retrieval that falls back to Static Sink + window when too few
+                               frames were detected ([digest] weaknesses, point 5)
+  bank_update_gated            bank refresh after the freeze, gated on fingerprint distance
+  bank_update_decay /          decay-weighted continuous writes after the freeze (moving
+    bank_blend_kv              average of the nearest entry's fingerprint and K/V)
+                               ([digest] weaknesses, point 3)
+  stream_decisions_policy      the decision sequence of a stream under one of these policies
 
 Readings taken where the sources are silent (each is repeated at its function):
 
@@ -64,6 +71,9 @@ __all__ = [
     "query_positions", "rope_angles", "rope_rotate", "attention", "attention_probs",
     "kv_append", "dyn_copy", "bank_store", "fingerprint", "retrieve", "retrieval_margin",
     "bank_objective", "bank_update", "bank_margin", "valid_mask", "stream_decisions",
+    "detected_frames", "retrieve_fallback", "fingerprint_distances", "bank_update_gated",
+    "gate_margin", "nearest_entry", "nearest_margin", "blend_weights", "bank_update_decay",
+    "bank_blend_kv", "stream_decisions_policy",
 ]
 
 # Slot identifiers; bit i of a validity mask refers to slot i.
@@ -505,4 +515,181 @@ def stream_decisions(phis, M: int = 5, write_blocks: int = 20):
         out.append(dict(r=r, score=sc, src=src, copy=copy, dyn_src=dyn_src, action=action,
                         count=count, bank_src=bank_src.copy(), retrieval_margin=rm,
                         bank_margin=bm))
+    return out
+
+
+# --------------------------------------------------------------------------------------------
+# bank policy variants ([digest] weaknesses, points 3 and 5: fixes the digest proposes for a
+# frozen bank and for failed pose detection)
+# --------------------------------------------------------------------------------------------
+
+def detected_frames(ok) -> int:
+    """Number of frames of a block whose pose detection succeeded."""
+    return int(sum(1 for x in ok if x))
+
+
+def retrieve_fallback(phi_b, ok, min_detected: int, bank_phi, bank_src, count: int,
+                      exclude: int):
+    """Retrieval with the fallback to the Static Sink + window cache.
+
+    [digest] weaknesses, point 5: the fingerprint depends on detection quality and failed frames
+    are zero-filled, so retrieval degrades under occlusion; one proposed fix is to fall back to
+    the conservative cache of Static Sink + window when detection is missing.  Reading: when
+    fewer than ``min_detected`` of the block's frames were detected, no entry is retrieved
+    (r = -1, the dynamic sink is empty for the block); otherwise this is ``retrieve``.
+    ``min_detected = 0`` never falls back.
+    """
+    if detected_frames(ok) < min_detected:
+        return -1, -np.inf
+    return retrieve(phi_b, bank_phi, bank_src, count, exclude)
+
+
+def fingerprint_distances(phi_b, bank_phi, count: int) -> np.ndarray:
+    """Euclidean distance ||phi_b - phi_i|| to every entry in use (float64)."""
+    phi_b = np.asarray(phi_b, dtype=np.float64)
+    return np.array([math.sqrt(float(np.sum((np.asarray(bank_phi[i], dtype=np.float64)
+                                             - phi_b) ** 2))) for i in range(int(count))])
+
+
+def bank_update_gated(bank_phi, bank_src, count: int, M: int, phi_b, b: int,
+                      write_blocks: int, gate: float):
+    """Diversity update with a refresh gated on fingerprint distance.
+
+    [digest] weaknesses, point 3: a bank frozen after the first 20 blocks misses states that
+    appear later; one proposed fix is to trigger a bank refresh gated on fingerprint distance.
+    Reading: for b < write_blocks this is ``bank_update``; afterwards the bank stays frozen
+    unless the block is farther than ``gate`` from every entry (min_i ||phi_b - phi_i|| >
+    gate), in which case the diversity rule of ``bank_update`` runs for it (insert while the
+    bank has room, else keep / replace j, whichever gives the least mean similarity).
+    Returns ``(action, bank_phi', bank_src', count')``.
+    """
+    if b < write_blocks:
+        return bank_update(bank_phi, bank_src, count, M, phi_b, b, write_blocks)
+    dist = fingerprint_distances(phi_b, bank_phi, count)
+    if count > 0 and not float(dist.min()) > gate:
+        return -1, np.array(bank_phi, dtype=np.float64, copy=True), np.array(bank_src, copy=True), count
+    return bank_update(bank_phi, bank_src, count, M, phi_b, b, b + 1)
+
+
+def gate_margin(phi_b, bank_phi, count: int, b: int, write_blocks: int, gate: float) -> float:
+    """|min distance - gate| (inf when the gate is not consulted)."""
+    if b < write_blocks or count == 0:
+        return math.inf
+    return abs(float(fingerprint_distances(phi_b, bank_phi, count).min()) - gate)
+
+
+def nearest_entry(phi_b, bank_phi, count: int):
+    """argmax_i phi_b . phi_i over the entries in use (ties to the lowest slot): ``(j, score)``,
+    ``(-1, -inf)`` for an empty bank."""
+    return retrieve(phi_b, bank_phi, np.full(max(int(count), 1), -1, dtype=np.int64), count,
+                    exclude=-2)
+
+
+def nearest_margin(phi_b, bank_phi, count: int) -> float:
+    return retrieval_margin(phi_b, bank_phi, np.full(max(int(count), 1), -1, dtype=np.int64),
+                            count, exclude=-2)
+
+
+def blend_weights(alpha: float):
+    """The float32 weights of a decayed write: (1 - alpha) for the entry, alpha for the block."""
+    a = np.float32(alpha)
+    return np.float32(np.float32(1.0) - a), a
+
+
+def bank_update_decay(bank_phi, bank_src, count: int, M: int, phi_b, b: int,
+                      write_blocks: int, alpha: float):
+    """Diversity update followed by decay-weighted continuous writes.
+
+    [digest] weaknesses, point 3: instead of freezing the bank after 20 blocks, allow
+    continuous writes with decaying weights.  Reading: for b < write_blocks this is
+    ``bank_update``; afterwards (alpha > 0) every block is written into the entry nearest to
+    it, j = argmax_i phi_b . phi_i, as an exponential moving average: the entry's fingerprint
+    becomes the l2-normalised (1 - alpha) phi_j + alpha phi_b and its K/V (1 - alpha) KV_j +
+    alpha KV_b (``bank_blend_kv``), so the weight of a write decays by (1 - alpha) with every
+    later write; src_j becomes b.  alpha = 0 keeps the bank frozen.
+    Returns ``(action, mode, bank_phi', bank_src', count')`` with mode "store" (a block's K/V
+    replaces an entry), "blend" or None.
+    """
+    if b < write_blocks:
+        action, bp, bs, c = bank_update(bank_phi, bank_src, count, M, phi_b, b, write_blocks)
+        return action, ("store" if action >= 0 else None), bp, bs, c
+    bank_phi = np.array(bank_phi, dtype=np.float64, copy=True)
+    bank_src = np.array(bank_src, copy=True)
+    if not alpha > 0.0 or count == 0:
+        return -1, None, bank_phi, bank_src, count
+    j, _ = nearest_entry(phi_b, bank_phi, count)
+    w_old, w_new = blend_weights(alpha)
+    t = float(w_old) * bank_phi[j] + float(w_new) * np.asarray(phi_b, dtype=np.float64)
+    n = math.sqrt(float(np.dot(t, t)))
+    bank_phi[j] = t / n if n > 0 else t
+    bank_src[j] = b
+    return j, "blend", bank_phi, bank_src, count
+
+
+def bank_blend_kv(cfg: dict, cache_kv, bank_kv, ring_slot: int, bank_slot: int, alpha: float):
+    """K/V of a decayed write: every element of bank entry ``bank_slot`` (all layers) becomes
+    bf16(fl32(fl32(w_old * x) + fl32(w_new * z))) with x the entry's value, z the block's clean
+    value in ring slot ``ring_slot`` and (w_old, w_new) = ``blend_weights(alpha)``: each product
+    and the sum rounded to float32 (no fused multiply-add), the result rounded to bf16 (nearest
+    even).  Returns the new bank as float64 holding bf16 values."""
+    import torch
+    a, e = slot_ranges(cfg)[SLOT_RING0 + ring_slot]
+    w_old, w_new = blend_weights(alpha)
+    x = np.asarray(bank_kv)[:, bank_slot].astype(np.float32)
+    z = np.asarray(cache_kv)[:, :, :, a:e, :].astype(np.float32)
+    y = (x * w_old).astype(np.float32) + (z * w_new).astype(np.float32)
+    y16 = torch.from_numpy(np.ascontiguousarray(y.astype(np.float32))).to(torch.bfloat16)
+    out = np.array(bank_kv, dtype=np.float64, copy=True)
+    out[:, bank_slot] = y16.to(torch.float64).numpy()
+    return out
+
+
+def stream_decisions_policy(phis, oks, M: int = 5, write_blocks: int = 20, policy: str = "frozen",
+                            alpha: float = 0.0, gate: float = 0.0, min_detected: int = 0):
+    """Decisions of a stream under a bank policy: "frozen" (the pages' rule, as
+    ``stream_decisions``), "decay" (``bank_update_decay`` with ``alpha``) or "gated"
+    (``bank_update_gated`` with ``gate``); retrieval falls back to Static Sink + window for
+    blocks with fewer than ``min_detected`` detected frames (``retrieve_fallback``).
+
+    Returns a list of dicts with keys r, score, src, copy, dyn_src, action, mode, count,
+    bank_src, bank_phi and the margins of the decisions taken (retrieval, bank, gate, nearest).
+    """
+    dim = len(phis[0])
+    bank_phi = np.zeros((M, dim), dtype=np.float64)
+    bank_src = np.full(M, -1, dtype=np.int64)
+    count = 0
+    dyn_src = -1
+    out = []
+    for b, (phi, ok) in enumerate(zip(phis, oks)):
+        fallback = detected_frames(ok) < min_detected
+        rm = math.inf if fallback else retrieval_margin(phi, bank_phi, bank_src, count, b - 1)
+        r, sc = retrieve_fallback(phi, ok, min_detected, bank_phi, bank_src, count, b - 1)
+        src = int(bank_src[r]) if r >= 0 else -1
+        copy = r >= 0 and src != dyn_src
+        dyn_src = src
+        bm = bank_margin(bank_phi, count, M, phi, b, write_blocks)
+        gm = nm = math.inf
+        if policy == "frozen":
+            action, bank_phi, bank_src, count = bank_update(bank_phi, bank_src, count, M, phi, b,
+                                                            write_blocks)
+            mode = "store" if action >= 0 else None
+        elif policy == "gated":
+            gm = gate_margin(phi, bank_phi, count, b, write_blocks, gate)
+            if b >= write_blocks:
+                opened = count == 0 or float(fingerprint_distances(phi, bank_phi, count).min()) > gate
+                bm = bank_margin(bank_phi, count, M, phi, 0, 1) if opened else math.inf
+            action, bank_phi, bank_src, count = bank_update_gated(bank_phi, bank_src, count, M,
+                                                                  phi, b, write_blocks, gate)
+            mode = "store" if action >= 0 else None
+        elif policy == "decay":
+            if b >= write_blocks and alpha > 0 and count > 0:
+                nm = nearest_margin(phi, bank_phi, count)
+            action, mode, bank_phi, bank_src, count = bank_update_decay(
+                bank_phi, bank_src, count, M, phi, b, write_blocks, alpha)
+        else:
+            raise ValueError(policy)
+        out.append(dict(r=r, score=sc, src=src, copy=copy, dyn_src=dyn_src, action=action,
+                        mode=mode, count=count, bank_src=bank_src.copy(),
+                        bank_phi=bank_phi.copy(), retrieval_margin=rm, bank_margin=bm,
+                        gate_margin=gm, nearest_margin=nm))
     return out
