@@ -191,6 +191,62 @@ int prsink_bank_update(const prsink_layout* layout, float* bank_phi, long long* 
                        int write_blocks, int* action_out, const void* cache_kv, void* bank_kv,
                        int n_layers, void* stream);
 
+/* ---- bank policy variants -------------------------------------------------------------
+ * [digest] weaknesses, point 3: a bank frozen after the first 20 blocks assumes the pose
+ * distribution is sampled at the start of the stream; proposed fixes are continuous writes
+ * with decaying weights and a refresh gated on fingerprint distance.  [digest] weaknesses,
+ * point 5: under failed detection retrieval degrades; a proposed fix is to fall back to the
+ * conservative Static Sink + window cache.  These calls implement those readings; the calls
+ * above implement the pages' own rule. */
+#define PRSINK_BANK_FROZEN 0       /* the pages' rule: diversity writes, then frozen        */
+#define PRSINK_BANK_DECAY  1       /* after the freeze: moving average into the nearest entry */
+#define PRSINK_BANK_GATED  2       /* after the freeze: diversity rule for far-away blocks   */
+
+#define PRSINK_BANK_MODE_NONE  0   /* mode word: nothing written                            */
+#define PRSINK_BANK_MODE_STORE 1   /* the block's fingerprint and K/V replace entry `action` */
+#define PRSINK_BANK_MODE_BLEND 2   /* entry `action` averaged with the block                */
+
+typedef struct prsink_bank_policy {
+  int kind;            /* PRSINK_BANK_FROZEN / _DECAY / _GATED                               */
+  int write_blocks;    /* the diversity rule runs for blocks b < write_blocks (20)           */
+  float alpha;         /* DECAY, in [0, 1]: weight of the block.  For b >= write_blocks the
+                          block goes into its nearest entry j = argmax_i phi_b . phi_i (ties
+                          to the lowest slot): phi_j <- l2-normalised((1-alpha) phi_j + alpha
+                          phi_b) (float64), every K/V element x of entry j (all layers) <-
+                          bf16(fl32(fl32(w_old x) + fl32(alpha z))), w_old = fl32(1 - alpha),
+                          z the block's clean K/V; src_j <- b.  alpha = 0 writes nothing.    */
+  float gate;          /* GATED: for b >= write_blocks the diversity rule runs for a block
+                          with min_i ||phi_b - phi_i||_2 > gate (float64), else nothing is
+                          written                                                            */
+} prsink_bank_policy;
+
+/* prsink_retrieve with the fallback to Static Sink + window: when fewer than `min_detected`
+ * (0..3) of the block's frames were detected (frame_ok: u8 [3] on the device, as given to
+ * prsink_fingerprint), no entry is retrieved: r = -1, *dyn_src = -1 (the dynamic sink is empty
+ * for the block's attention calls), *copy_out = 0.  Otherwise identical to prsink_retrieve.
+ * Errors: as prsink_retrieve; PRSINK_ERR_ARG for a null frame_ok or min_detected outside
+ * [0, 3]. */
+int prsink_retrieve_fallback(const prsink_layout* layout, const float* phi_b,
+                             const unsigned char* frame_ok, int min_detected,
+                             const float* bank_phi, const long long* bank_src,
+                             const int* bank_count, int M, long long exclude_block, int* r_out,
+                             float* score_out, int* copy_out, long long* dyn_src,
+                             const void* bank_kv, void* cache_kv, int n_layers, void* stream);
+
+/* prsink_bank_update under a policy.  For b < policy->write_blocks, and for every block with
+ * PRSINK_BANK_FROZEN, identical to prsink_bank_update with write_blocks = policy->write_blocks.
+ *   action_out  int32 scalar (written): the entry written, or -1
+ *   mode_out    int32 scalar (written, device, required): PRSINK_BANK_MODE_*; the K/V copies
+ *               that follow read it, so the decision stays on the device
+ *   cache_kv, bank_kv, n_layers: as prsink_bank_update; a store copies block b's clean K/V
+ *               (ring slot b mod R of every layer) into entry `action`, a blend averages it in.
+ * Errors: as prsink_bank_update; PRSINK_ERR_ARG for a null policy or mode_out, an unknown kind,
+ * alpha outside [0, 1], a non-finite gate or write_blocks < 0. */
+int prsink_bank_update_policy(const prsink_layout* layout, const prsink_bank_policy* policy,
+                              float* bank_phi, long long* bank_src, int* bank_count, int M,
+                              const float* phi_b, long long b, int* action_out, int* mode_out,
+                              const void* cache_kv, void* bank_kv, int n_layers, void* stream);
+
 /* Synchronise `stream`, then read and clear the status word of the current device:
  * PRSINK_OK, or PRSINK_ERR_TIMEOUT if a bounded wait of any kernel on this device (any
  * stream) ran out since the word was last cleared, or PRSINK_ERR_LAUNCH.  Only `stream` is

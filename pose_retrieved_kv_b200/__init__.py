@@ -10,5 +10,7 @@ from ._lib import (  # noqa: F401
     SLOT_STATIC, LIB_PATH, Layout, PRSinkError, exported_symbols, make_layout,
     prsink_attention, prsink_bank_update, prsink_debug_wait_timeout, prsink_fingerprint,
     prsink_kv_append, prsink_last_error, prsink_launch_count, prsink_layout_tokens,
-    prsink_retrieve, prsink_sync_status, prsink_version)
+    prsink_retrieve, prsink_sync_status, prsink_version, BANK_DECAY, BANK_FROZEN, BANK_GATED,
+    BANK_MODE_BLEND, BANK_MODE_NONE, BANK_MODE_STORE, BankPolicy, make_policy,
+    prsink_bank_update_policy, prsink_retrieve_fallback)
 from .stream import PRSinkStream, stream_valid_mask  # noqa: F401

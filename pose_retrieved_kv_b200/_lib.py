@@ -50,6 +50,25 @@ class Layout(ctypes.Structure):
                 ("block_index", ctypes.c_longlong), ("valid_mask", ctypes.c_uint)]
 
 
+BANK_FROZEN, BANK_DECAY, BANK_GATED = 0, 1, 2
+BANK_MODE_NONE, BANK_MODE_STORE, BANK_MODE_BLEND = 0, 1, 2
+_KINDS = {"frozen": BANK_FROZEN, "decay": BANK_DECAY, "gated": BANK_GATED}
+
+
+class BankPolicy(ctypes.Structure):
+    """Mirror of ``prsink_bank_policy``."""
+    _fields_ = [("kind", ctypes.c_int), ("write_blocks", ctypes.c_int),
+                ("alpha", ctypes.c_float), ("gate", ctypes.c_float)]
+
+
+def make_policy(kind="frozen", write_blocks: int = 20, alpha: float = 0.0,
+                gate: float = 0.0) -> BankPolicy:
+    pol = BankPolicy()
+    pol.kind = _KINDS[kind] if isinstance(kind, str) else int(kind)
+    pol.write_blocks, pol.alpha, pol.gate = int(write_blocks), float(alpha), float(gate)
+    return pol
+
+
 def make_layout(n_heads, head_dim, grid_h, grid_w, frames_per_block=3, ref_frames=1,
                 ring_slots=3, rope_mode=3, rope_split=(44, 42, 42), rope_base=10000.0,
                 block_index=0, valid_mask=0xFFFFFFFF, **_ignored) -> Layout:
@@ -83,6 +102,10 @@ def _load():
         "prsink_fingerprint": ([vp, vp, vp, vp], i),
         "prsink_retrieve": ([lp, vp, vp, vp, vp, i, ll, vp, vp, vp, vp, vp, vp, i, vp], i),
         "prsink_bank_update": ([lp, vp, vp, vp, i, vp, ll, i, vp, vp, vp, i, vp], i),
+        "prsink_retrieve_fallback": ([lp, vp, vp, i, vp, vp, vp, i, ll, vp, vp, vp, vp, vp, vp,
+                                      i, vp], i),
+        "prsink_bank_update_policy": ([lp, ctypes.POINTER(BankPolicy), vp, vp, vp, i, vp, ll,
+                                       vp, vp, vp, vp, i, vp], i),
         "prsink_sync_status": ([vp], i),
         "prsink_debug_wait_timeout": ([ll, vp], i),
     }
@@ -99,7 +122,8 @@ _lib = _load()
 def exported_symbols() -> list:
     return ["prsink_version", "prsink_last_error", "prsink_launch_count", "prsink_layout_tokens",
             "prsink_attention", "prsink_kv_append", "prsink_fingerprint", "prsink_retrieve",
-            "prsink_bank_update", "prsink_sync_status", "prsink_debug_wait_timeout"]
+            "prsink_bank_update", "prsink_sync_status", "prsink_debug_wait_timeout",
+            "prsink_retrieve_fallback", "prsink_bank_update_policy"]
 
 
 def _check(rc: int, fn: str):
@@ -233,6 +257,39 @@ def prsink_bank_update(layout: Optional[Layout], bank_phi, bank_src, bank_count,
         _ptr(cache_kv, "cache_kv", torch.bfloat16, n_cache),
         _ptr(bank_kv, "bank_kv", torch.bfloat16, n_bank), int(n_layers), _stream(stream))
     _check(rc, "prsink_bank_update")
+
+
+def prsink_retrieve_fallback(layout: Optional[Layout], phi_b, frame_ok, min_detected: int,
+                             bank_phi, bank_src, bank_count, M: int, exclude_block: int, r_out,
+                             score_out, copy_out, dyn_src, bank_kv=None, cache_kv=None,
+                             n_layers: int = 0, stream=None):
+    n_bank, n_cache = _kv_sizes(layout, M, n_layers, bank_kv, cache_kv)
+    rc = _lib.prsink_retrieve_fallback(
+        ctypes.byref(layout) if layout is not None else None,
+        _ptr(phi_b, "phi_b", torch.float32, FP_DIM), _ptr(frame_ok, "frame_ok", torch.uint8, 3),
+        int(min_detected), _ptr(bank_phi, "bank_phi", torch.float32, M * FP_DIM),
+        _ptr(bank_src, "bank_src", torch.int64, M), _ptr(bank_count, "bank_count", torch.int32, 1),
+        int(M), int(exclude_block), _ptr(r_out, "r_out", torch.int32, 1),
+        _ptr(score_out, "score_out", torch.float32, 1),
+        _ptr(copy_out, "copy_out", torch.int32, 1), _ptr(dyn_src, "dyn_src", torch.int64, 1),
+        _ptr(bank_kv, "bank_kv", torch.bfloat16, n_bank),
+        _ptr(cache_kv, "cache_kv", torch.bfloat16, n_cache), int(n_layers), _stream(stream))
+    _check(rc, "prsink_retrieve_fallback")
+
+
+def prsink_bank_update_policy(layout: Optional[Layout], policy: BankPolicy, bank_phi, bank_src,
+                              bank_count, M: int, phi_b, b: int, action_out, mode_out,
+                              cache_kv=None, bank_kv=None, n_layers: int = 0, stream=None):
+    n_bank, n_cache = _kv_sizes(layout, M, n_layers, bank_kv, cache_kv)
+    rc = _lib.prsink_bank_update_policy(
+        ctypes.byref(layout) if layout is not None else None, ctypes.byref(policy),
+        _ptr(bank_phi, "bank_phi", torch.float32, M * FP_DIM),
+        _ptr(bank_src, "bank_src", torch.int64, M), _ptr(bank_count, "bank_count", torch.int32, 1),
+        int(M), _ptr(phi_b, "phi_b", torch.float32, FP_DIM), int(b),
+        _ptr(action_out, "action_out", torch.int32, 1), _ptr(mode_out, "mode_out", torch.int32, 1),
+        _ptr(cache_kv, "cache_kv", torch.bfloat16, n_cache),
+        _ptr(bank_kv, "bank_kv", torch.bfloat16, n_bank), int(n_layers), _stream(stream))
+    _check(rc, "prsink_bank_update_policy")
 
 
 def prsink_sync_status(stream=None) -> int:

@@ -3,9 +3,13 @@
 //     them, into one slot of the head-major caches [H][T][d] (a transpose at 2*d-byte rows);
 //   * the dynamic-sink fill (bank entry r -> dynamic slot of every layer) and the bank store
 //     (ring slot of block b -> bank entry `action` of every layer), both predicated on a
-//     decision that stays in device memory.
+//     decision that stays in device memory;
+//   * the decayed bank write, bank entry <- (1 - alpha) entry + alpha block, element-wise in
+//     float32 rounded to bf16, predicated the same way.
 // Every thread moves 16-byte chunks; a 256-byte head row is one 16-lane run, so reads and
 // writes are fully coalesced without staging through shared memory.
+#include <cuda_bf16.h>
+
 #include "prsink_internal.cuh"
 
 namespace prsink {
@@ -73,8 +77,8 @@ append_rows_kernel(const uint4* __restrict__ k_new, const uint4* __restrict__ v_
 }
 
 // Segment copy: segment y (one (layer, k|v, head) run of `seg_chunks` contiguous chunks) from
-// src + y-dependent offset to dst + y-dependent offset.  Runs only if *flag != 0 (flag may be
-// null) and *sel >= 0; *sel picks the bank entry on the bank side.
+// src + y-dependent offset to dst + y-dependent offset.  Runs only if *sel >= 0 and, when flag
+// is given, *flag == want; *sel picks the bank entry on the bank side.
 struct SegCopy {
   const uint4* src;
   uint4* dst;
@@ -86,9 +90,9 @@ struct SegCopy {
 };
 
 __global__ void __launch_bounds__(kCopyThreads)
-seg_copy_kernel(SegCopy p, const int* __restrict__ sel, const int* __restrict__ flag) {
+seg_copy_kernel(SegCopy p, const int* __restrict__ sel, const int* __restrict__ flag, int want) {
   const int s = *sel;
-  if (s < 0 || (flag && *flag == 0)) return;
+  if (s < 0 || (flag && *flag != want)) return;
   const uint32_t y = blockIdx.y;               // = (layer*2 + kv)*H + head
   const uint32_t head = y % p.H;
   const uint32_t lk = y / p.H;
@@ -116,6 +120,46 @@ seg_copy_kernel(SegCopy p, const int* __restrict__ sel, const int* __restrict__ 
   }
 }
 
+// w_old * x + w_new * z for the 8 bf16 of a chunk: each product and the sum rounded to
+// float32 (no fused multiply-add), the result rounded to bf16 (nearest even).
+__device__ __forceinline__ uint32_t blend_pair(uint32_t x, uint32_t z, float w_old, float w_new) {
+  const float lo = __fadd_rn(__fmul_rn(w_old, __uint_as_float(x << 16)),
+                             __fmul_rn(w_new, __uint_as_float(z << 16)));
+  const float hi = __fadd_rn(__fmul_rn(w_old, __uint_as_float(x & 0xFFFF0000u)),
+                             __fmul_rn(w_new, __uint_as_float(z & 0xFFFF0000u)));
+  __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&b);
+}
+
+// Decayed bank write: dst (bank entry, read and written) <- w_old * dst + w_new * src (ring
+// slot), same segments and predicate as seg_copy_kernel.
+__global__ void __launch_bounds__(kCopyThreads)
+seg_blend_kernel(SegCopy p, const int* __restrict__ sel, const int* __restrict__ flag, int want,
+                 float w_old, float w_new) {
+  const int s = *sel;
+  if (s < 0 || (flag && *flag != want)) return;
+  const uint32_t y = blockIdx.y;
+  const uint32_t head = y % p.H;
+  const uint32_t lk = y / p.H;
+  const uint32_t kv = lk & 1u;
+  const uint32_t layer = lk >> 1;
+  const uint4* __restrict__ src = p.src + p.src_base + layer * p.src_layer + kv * p.src_kv +
+                                  head * p.src_head + static_cast<uint64_t>(s) * p.src_sel;
+  uint4* __restrict__ dst = p.dst + p.dst_base + layer * p.dst_layer + kv * p.dst_kv +
+                            head * p.dst_head + static_cast<uint64_t>(s) * p.dst_sel;
+  const uint64_t stride = static_cast<uint64_t>(gridDim.x) * kCopyThreads;
+  for (uint64_t i = static_cast<uint64_t>(blockIdx.x) * kCopyThreads + threadIdx.x;
+       i < p.seg_chunks; i += stride) {
+    const uint4 z = __ldcs(src + i);
+    uint4 x = dst[i];
+    x.x = blend_pair(x.x, z.x, w_old, w_new);
+    x.y = blend_pair(x.y, z.y, w_old, w_new);
+    x.z = blend_pair(x.z, z.z, w_old, w_new);
+    x.w = blend_pair(x.w, z.w, w_old, w_new);
+    dst[i] = x;
+  }
+}
+
 static int grid_for(uint64_t chunks) {
   uint64_t g = (chunks + kCopyThreads * kCopyUnroll - 1) / (kCopyThreads * kCopyUnroll);
   if (g < 1) g = 1;
@@ -124,10 +168,12 @@ static int grid_for(uint64_t chunks) {
 }
 
 // Launch the predicated copy between bank entry *sel and cache slot `slot` of every layer.
-// to_cache = true: bank -> cache (dynamic-sink fill); false: cache -> bank (bank store).
+// to_cache = true: bank -> cache (dynamic-sink fill); false: cache -> bank (bank store, or the
+// decayed write when blend_alpha >= 0).  Runs iff *sel >= 0 and (flag null or *flag == want).
 int launch_bank_cache_copy(const prsink_layout* L, const Geometry& g, int M, int n_layers,
                            const void* bank_kv, const void* cache_kv, bool to_cache, int slot,
-                           const int* sel, const int* flag, cudaStream_t st) {
+                           const int* sel, const int* flag, int want, cudaStream_t st,
+                           float blend_alpha) {
   const uint64_t C = static_cast<uint64_t>(L->head_dim) * 2 / 16;   // chunks per row
   const uint64_t H = L->n_heads;
   // cache_kv [layers][2][H][T][d]; bank_kv [layers][M][2][H][L_blk][d]
@@ -170,7 +216,13 @@ int launch_bank_cache_copy(const prsink_layout* L, const Geometry& g, int M, int
   if (gx > gmax) gx = gmax;
   if (gx < 1) gx = 1;
   dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(segs));
-  seg_copy_kernel<<<grid, kCopyThreads, 0, st>>>(p, sel, flag);
+  if (blend_alpha >= 0.f) {
+    const float w_new = blend_alpha;
+    const float w_old = 1.0f - w_new;          // float32 subtraction, as the weights are defined
+    seg_blend_kernel<<<grid, kCopyThreads, 0, st>>>(p, sel, flag, want, w_old, w_new);
+  } else {
+    seg_copy_kernel<<<grid, kCopyThreads, 0, st>>>(p, sel, flag, want);
+  }
   count_launch();
   return check_launch("bank/cache copy");
 }

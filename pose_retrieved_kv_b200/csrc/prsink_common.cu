@@ -116,7 +116,7 @@ using namespace prsink;
 
 extern "C" {
 
-int prsink_version(void) { return 1; }
+int prsink_version(void) { return 2; }
 
 const char* prsink_last_error(void) { return g_err; }
 

@@ -44,9 +44,15 @@ class PRSinkStream:
     """
 
     def __init__(self, cfg: dict, n_layers: int, M: int = 5, write_blocks: int = 20,
-                 device="cuda"):
+                 device="cuda", policy: str = "frozen", alpha: float = 0.0, gate: float = 0.0,
+                 min_detected: int = 0):
+        """``policy``, ``alpha``, ``gate``: the bank policy (the pages' frozen bank, or one of
+        the variants of ``prsink_bank_update_policy``); ``min_detected`` > 0 makes retrieval
+        fall back to Static Sink + window for blocks with fewer detected frames."""
         self.cfg = dict(cfg)
         self.n_layers, self.M, self.write_blocks = int(n_layers), int(M), int(write_blocks)
+        self.policy = L.make_policy(policy, write_blocks, alpha, gate)
+        self.min_detected = int(min_detected)
         self.R = int(cfg["ring_slots"])
         lay = L.make_layout(**{**self.cfg, "block_index": 0, "valid_mask": 0})
         self.L_f, self.L_blk, self.L_ref, self.T = L.prsink_layout_tokens(lay)
@@ -64,6 +70,8 @@ class PRSinkStream:
         self.score = torch.zeros(1, dtype=torch.float32, device=dev)
         self.copied = torch.zeros(1, dtype=torch.int32, device=dev)
         self.action = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.mode = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.frame_ok = torch.ones(3, dtype=torch.uint8, device=dev)
         self.b = 0
 
     def reset(self):
@@ -91,6 +99,13 @@ class PRSinkStream:
     def begin_block(self, kp, frame_ok, stream=None):
         """Fingerprint (kp f32 [3][62][3], frame_ok u8 [3], on the device) and retrieval."""
         L.prsink_fingerprint(kp, frame_ok, self.phi, stream)
+        if self.min_detected > 0:
+            L.prsink_retrieve_fallback(self.layout(), self.phi, frame_ok, self.min_detected,
+                                       self.bank_phi, self.bank_src, self.bank_count, self.M,
+                                       self.b - 1, self.r, self.score, self.copied,
+                                       self.dyn_src, self.bank_kv, self.cache_kv,
+                                       self.n_layers, stream)
+            return
         L.prsink_retrieve(self.layout(), self.phi, self.bank_phi, self.bank_src,
                           self.bank_count, self.M, self.b - 1, self.r, self.score, self.copied,
                           self.dyn_src, self.bank_kv, self.cache_kv, self.n_layers, stream)
@@ -109,9 +124,15 @@ class PRSinkStream:
     def end_block(self, stream=None, check: bool = False):
         """Bank update with the clean K/V of block b, then advance to block b+1.  With
         ``check`` the stream is synchronised and a device timeout raises."""
-        L.prsink_bank_update(self.layout(), self.bank_phi, self.bank_src, self.bank_count,
-                             self.M, self.phi, self.b, self.write_blocks, self.action,
-                             self.cache_kv, self.bank_kv, self.n_layers, stream)
+        if self.policy.kind == L.BANK_FROZEN:
+            L.prsink_bank_update(self.layout(), self.bank_phi, self.bank_src, self.bank_count,
+                                 self.M, self.phi, self.b, self.write_blocks, self.action,
+                                 self.cache_kv, self.bank_kv, self.n_layers, stream)
+        else:
+            L.prsink_bank_update_policy(self.layout(), self.policy, self.bank_phi,
+                                        self.bank_src, self.bank_count, self.M, self.phi,
+                                        self.b, self.action, self.mode, self.cache_kv,
+                                        self.bank_kv, self.n_layers, stream)
         self.b += 1
         if check:
             self.check_status(stream)
