@@ -112,6 +112,48 @@ int prsink_attention(const prsink_layout* layout, const void* q, const void* k_c
                      const void* v_cache, void* out, float* lse, const long long* dyn_src,
                      void* stream);
 
+/* Rotated copy of the sink keys, for prsink_attention_fused.
+ *
+ * [digest] weaknesses, point 2: reuse cached work to cut the repeated computation of the Ref and
+ * Static Sinks.  Within a block the positions of every slot but the current block's stay fixed
+ * (ring slots move one rank per block), so their keys can be rotated once per (block, layer)
+ * instead of by every attention pass and every query tile.  This call rotates, for every head,
+ * the raw keys of the slots in `slot_mask` (bit i = slot i) that hold data (valid_mask) at the
+ * positions they have while block `layout->block_index` is generated, into k_rot.  The current
+ * block's ring slot (b mod R) is never rotated (the fused attention reads that block from
+ * k_new).  Rows of other slots sharing a 128-row tile with a rotated slot are rewritten with
+ * their own rotation (identical for slots whose positions did not change).
+ *   k_cache   bf16 [H][T][d]  raw keys (read)
+ *   k_rot     bf16 [H][T][d]  rotated keys (written); a buffer of its own
+ *   slot_mask slots to rotate.  A ring slot must be rotated at every block (its rank changes);
+ *             ref / static / dynamic only when written (their positions never change).
+ *   dyn_flag  int32 scalar or NULL: if given and 0, the dynamic slot is skipped (e.g. the
+ *             retrieval's copy_out: the slot was not refilled)
+ *   dyn_src   int64 scalar or NULL: if given and < 0 the dynamic slot is empty (skipped)
+ * The rotation is the attention kernel's own (float32 with cos/sin tables from float64), so the
+ * rotated keys equal those prsink_attention computes internally, bit for bit.
+ * Errors: PRSINK_ERR_ARG, PRSINK_ERR_ALIGN, PRSINK_ERR_UNSUPPORTED, PRSINK_ERR_LAUNCH. */
+int prsink_rotate_sinks(const prsink_layout* layout, const void* k_cache, void* k_rot,
+                        unsigned slot_mask, const int* dyn_flag, const long long* dyn_src,
+                        void* stream);
+
+/* Attention of the current block with its Clean KV Update / per-pass append folded in.
+ *
+ * [digest] weaknesses, point 2 (Clean KV Update is 24.39 % of the time; cache reuse of the
+ * sinks).  Equivalent to prsink_kv_append(k_new, v_new -> ring slot b mod R of k_cache /
+ * v_cache) followed by prsink_attention(q, k_cache, v_cache), with the keys of every other slot
+ * read already rotated from k_rot (prsink_rotate_sinks of this block, kept current by the
+ * caller) instead of being rotated here.  The current block's keys are read from k_new, rotated
+ * at the current block's positions and attended whatever valid_mask says about its slot; the
+ * raw k_new / v_new rows are stored into the ring slot by the same launch.
+ *   q, out, lse, dyn_src as prsink_attention;  k_new, v_new bf16 [L_blk][H][d] (token-major);
+ *   k_rot bf16 [H][T][d] (read);  k_cache, v_cache bf16 [H][T][d]: V of the other slots read,
+ *   the ring slot's K and V rows written (no other byte).
+ * Errors: as prsink_attention. */
+int prsink_attention_fused(const prsink_layout* layout, const void* q, const void* k_new,
+                           const void* v_new, const void* k_rot, void* k_cache, void* v_cache,
+                           void* out, float* lse, const long long* dyn_src, void* stream);
+
 /* Clean KV Update / per-pass append: write one slot's raw K and V into the caches.
  *
  * [digest] pipeline, inference clause: KV_cache <- KV_cache U Forward(z^0_b, t=0, C) is

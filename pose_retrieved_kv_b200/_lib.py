@@ -102,6 +102,8 @@ def _load():
         "prsink_fingerprint": ([vp, vp, vp, vp], i),
         "prsink_retrieve": ([lp, vp, vp, vp, vp, i, ll, vp, vp, vp, vp, vp, vp, i, vp], i),
         "prsink_bank_update": ([lp, vp, vp, vp, i, vp, ll, i, vp, vp, vp, i, vp], i),
+        "prsink_attention_fused": ([lp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp], i),
+        "prsink_rotate_sinks": ([lp, vp, vp, ctypes.c_uint, vp, vp, vp], i),
         "prsink_retrieve_fallback": ([lp, vp, vp, i, vp, vp, vp, i, ll, vp, vp, vp, vp, vp, vp,
                                       i, vp], i),
         "prsink_bank_update_policy": ([lp, ctypes.POINTER(BankPolicy), vp, vp, vp, i, vp, ll,
@@ -123,7 +125,8 @@ def exported_symbols() -> list:
     return ["prsink_version", "prsink_last_error", "prsink_launch_count", "prsink_layout_tokens",
             "prsink_attention", "prsink_kv_append", "prsink_fingerprint", "prsink_retrieve",
             "prsink_bank_update", "prsink_sync_status", "prsink_debug_wait_timeout",
-            "prsink_retrieve_fallback", "prsink_bank_update_policy"]
+            "prsink_retrieve_fallback", "prsink_bank_update_policy", "prsink_attention_fused",
+            "prsink_rotate_sinks"]
 
 
 def _check(rc: int, fn: str):
@@ -205,6 +208,35 @@ def prsink_attention(layout: Layout, q, k_cache, v_cache, out, lse=None, dyn_src
         _ptr(lse, "lse", torch.float32, H * lblk), _ptr(dyn_src, "dyn_src", torch.int64, 1),
         _stream(stream))
     _check(rc, "prsink_attention")
+
+
+def prsink_attention_fused(layout: Layout, q, k_new, v_new, k_rot, k_cache, v_cache, out,
+                           lse=None, dyn_src=None, stream=None):
+    _, lblk, _, T = prsink_layout_tokens(layout)
+    H, d = layout.n_heads, layout.head_dim
+    rc = _lib.prsink_attention_fused(
+        ctypes.byref(layout), _ptr(q, "q", torch.bfloat16, lblk * H * d),
+        _ptr(k_new, "k_new", torch.bfloat16, lblk * H * d),
+        _ptr(v_new, "v_new", torch.bfloat16, lblk * H * d),
+        _ptr(k_rot, "k_rot", torch.bfloat16, H * T * d),
+        _ptr(k_cache, "k_cache", torch.bfloat16, H * T * d),
+        _ptr(v_cache, "v_cache", torch.bfloat16, H * T * d),
+        _ptr(out, "out", torch.bfloat16, lblk * H * d),
+        _ptr(lse, "lse", torch.float32, H * lblk), _ptr(dyn_src, "dyn_src", torch.int64, 1),
+        _stream(stream))
+    _check(rc, "prsink_attention_fused")
+
+
+def prsink_rotate_sinks(layout: Layout, k_cache, k_rot, slot_mask: int, dyn_flag=None,
+                        dyn_src=None, stream=None):
+    _, _, _, T = prsink_layout_tokens(layout)
+    H, d = layout.n_heads, layout.head_dim
+    rc = _lib.prsink_rotate_sinks(
+        ctypes.byref(layout), _ptr(k_cache, "k_cache", torch.bfloat16, H * T * d),
+        _ptr(k_rot, "k_rot", torch.bfloat16, H * T * d), int(slot_mask) & 0xFFFFFFFF,
+        _ptr(dyn_flag, "dyn_flag", torch.int32, 1), _ptr(dyn_src, "dyn_src", torch.int64, 1),
+        _stream(stream))
+    _check(rc, "prsink_rotate_sinks")
 
 
 def prsink_kv_append(layout: Layout, k_new, v_new, k_cache, v_cache, dest_slot: int,

@@ -22,6 +22,7 @@
 #include <cuda_bf16.h>
 
 #include <cmath>
+#include <initializer_list>
 #include <mutex>
 
 #include "prsink_internal.cuh"
@@ -61,14 +62,27 @@ struct Params {
   const long long* dyn_src;
   int* status;
   unsigned long long timeout_ns;
+  // fused form (the current block read from k_new / v_new and stored into its ring slot)
+  int cur_slot;                         // ring slot of the current block (slot id), or -1
+  int n_cur_tiles;                      // key tiles of the current block
+  // rotation pass (prsink_rotate_sinks): slots whose rows are rotated into k_rot
+  unsigned rot_mask;
+  const int* rot_dyn_flag;              // dynamic slot rotated only if *flag != 0 (nullable)
 };
+
+// Entries of the per-CTA tile list: a key tile index and what the roles do with it.
+constexpr uint16_t kTileIdx = 0x03FF;   // tile index (sink tiles: rows idx*BN..; current: tokens)
+constexpr uint16_t kTileVfix = 1u << 12;   // the rotation warps touch V before the P.V MMA
+constexpr uint16_t kTileStore = 1u << 13;  // this CTA stores the raw tile into the ring slot
+constexpr uint16_t kTileNew = 1u << 14;    // current-block tile (from k_new / v_new)
+constexpr uint16_t kTileMask = 1u << 15;   // some columns are masked (boundary or ragged tile)
 
 enum Bar {
   B_QFULL = 0, B_QREADY = 1,
   B_KFULL = 2, B_KREADY = 4, B_KEMPTY = 6,
   B_VFULL = 8, B_VFIX = 10, B_VEMPTY = 12,
   B_SFULL = 14, B_PFULL = 16, B_ODONE = 18,
-  B_FINAL = 20, B_COUNT = 21
+  B_FINAL = 20, B_KSTORED = 21, B_COUNT = 22
 };
 
 template <int D>
@@ -276,11 +290,79 @@ __device__ __forceinline__ void rotate_row(uint8_t* tile, int r, int frame, int 
   }
 }
 
+// RoPE tables in shared memory at `tabp`: cos / sin of pos * base^(-2j/d_axis), computed in
+// double (the angle reduced exactly by sincospi) and stored as float.  RT > 0 (the 44/42/42
+// split): grouped records per (axis, position, pair group): float4 (cos, cos', sin, sin') and
+// float2 (-sin, -sin').  RT == 0: float2 (cos, sin) per [position][pair] (3-D: t, h, w axes;
+// 1-D: the angle of the frame offset, then of the in-frame token).
 template <int D, int RT, int RH>
+__device__ void build_rope_tables(uint8_t* tabp, const Params& p, int tid, int nthr) {
+  float4* gcs = reinterpret_cast<float4*>(tabp);            // grouped tables (RT > 0)
+  float2* tab = reinterpret_cast<float2*>(tabp);             // [position][pair] (RT == 0)
+  using GR = Groups<(RT > 0 ? RT : 22), (RT > 0 ? RH : 21)>;
+  const int g_count = p.n_frames * GR::GT + p.grid_h * GR::GH + p.grid_w * GR::GW;
+  float2* gns = reinterpret_cast<float2*>(gcs + g_count);
+  if constexpr (RT > 0) {
+    const int offH = p.n_frames * GR::GT, offW = offH + p.grid_h * GR::GH;
+    for (int e = tid; e < g_count; e += nthr) {
+      int pos, g, na;
+      if (e < offH) { pos = e / GR::GT; g = e % GR::GT; na = RT; }
+      else if (e < offW) { pos = (e - offH) / GR::GH; g = (e - offH) % GR::GH; na = RH; }
+      else { pos = (e - offW) / GR::GW; g = (e - offW) % GR::GW; na = GR::RW; }
+      double sn[2] = {0.0, 0.0}, cs[2] = {1.0, 1.0};
+      const bool w_axis = e >= offW;
+#pragma unroll
+      for (int l = 0; l < 2; ++l) {
+        // t, h: record g holds pairs (2g, 2g+1); w: record 0 holds pair 0, record g >= 1
+        // holds pairs (2g-1, 2g)
+        const int jj = w_axis ? (g == 0 ? (l == 0 ? 0 : na) : 2 * g - 1 + l) : 2 * g + l;
+        if (jj < na) {
+          const double turns = static_cast<double>(pos) *
+                               exp2(-(2.0 * jj / (2 * na)) * p.log2_base) * 0.31830988618379067154;
+          sincospi(turns, &sn[l], &cs[l]);
+        }
+      }
+      gcs[e] = make_float4(static_cast<float>(cs[0]), static_cast<float>(cs[1]),
+                           static_cast<float>(sn[0]), static_cast<float>(sn[1]));
+      gns[e] = make_float2(-static_cast<float>(sn[0]), -static_cast<float>(sn[1]));
+    }
+  }
+  // Layout [position][pair j]; 3-D: t (frames), h (grid rows), w (grid columns); 1-D: angle
+  // of the frame offset frame*L_f, then of the in-frame token index.
+  for (int e = tid; RT == 0 && e < p.tab_entries; e += nthr) {
+    int pos, j, da;
+    if (p.rope_mode == 3) {
+      if (e < p.tab_h_off) { pos = e / p.rd[0]; j = e % p.rd[0]; da = 2 * p.rd[0]; }
+      else if (e < p.tab_w_off) { const int f = e - p.tab_h_off; pos = f / p.rd[1]; j = f % p.rd[1]; da = 2 * p.rd[1]; }
+      else { const int f = e - p.tab_w_off; pos = f / p.rd[2]; j = f % p.rd[2]; da = 2 * p.rd[2]; }
+    } else {
+      da = D;
+      if (e < p.tab_h_off) { pos = (e / (D / 2)) * p.L_f; j = e % (D / 2); }
+      else { const int f = e - p.tab_h_off; pos = f / (D / 2); j = f % (D / 2); }
+    }
+    // angle / pi, so that the reduction of the argument is exact (sincospi)
+    const double turns = static_cast<double>(pos) * exp2(-(2.0 * j / da) * p.log2_base) *
+                         0.31830988618379067154;
+    double sn, cs;
+    sincospi(turns, &sn, &cs);
+    tab[e] = make_float2(static_cast<float>(cs), static_cast<float>(sn));
+  }
+}
+
+// kFused = false: every key from the slot-indexed raw caches (tm_k, tm_v), rotated here.
+// kFused = true: keys of every slot but the current block's from the rotated copy (tm_k =
+// k_rot, already rotated at this block's positions; tm_v = v_cache); the current block's keys
+// and values from k_new / v_new (tm_kn, tm_vn), rotated here, and also stored raw into their
+// ring slot (tm_ks, tm_vs: maps over that slot of k_cache / v_cache), each tile by one CTA.
+template <int D, int RT, int RH, bool kFused>
 __global__ void __launch_bounds__(kThreads, 1)
 prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
                         const __grid_constant__ CUtensorMap tm_k,
-                        const __grid_constant__ CUtensorMap tm_v, const Params p) {
+                        const __grid_constant__ CUtensorMap tm_v,
+                        const __grid_constant__ CUtensorMap tm_kn,
+                        const __grid_constant__ CUtensorMap tm_vn,
+                        const __grid_constant__ CUtensorMap tm_ks,
+                        const __grid_constant__ CUtensorMap tm_vs, const Params p) {
   using LY = Layout<D>;
   extern __shared__ uint8_t dsmem[];
   __shared__ __align__(8) uint64_t bars[B_COUNT];
@@ -288,7 +370,7 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
   __shared__ AbortState ab;
   __shared__ unsigned vmask_s;
   __shared__ uint8_t tile_flag[kMaxTiles];       // bit 0: holds a valid key, bit 1: boundary
-  __shared__ uint16_t tile_list[kMaxTiles];      // live tiles in order; bit 15: boundary tile
+  __shared__ uint16_t tile_list[kMaxTiles];      // live tiles in order (kTile* bits)
   __shared__ int n_live_s;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -317,9 +399,11 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
       mbar_init(bar(B_ODONE + s), 1);
     }
     mbar_init(bar(B_FINAL), 1);
+    mbar_init(bar(B_KSTORED), 1);
     ab.flag = 0;
     unsigned vm = p.valid_mask;
     if (p.dyn_src && *p.dyn_src < 0) vm &= ~(1u << PRSINK_SLOT_DYNAMIC);
+    if (kFused) vm &= ~(1u << p.cur_slot);        // its keys come from k_new instead
     vmask_s = vm;
     fence_barrier_init();
   }
@@ -331,61 +415,21 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
     prefetch_tmap(&tm_q);
     prefetch_tmap(&tm_k);
     prefetch_tmap(&tm_v);
+    if (kFused) {
+      prefetch_tmap(&tm_kn);
+      prefetch_tmap(&tm_vn);
+    }
   }
   if (warp == kMmaWarp) {
     tmem_alloc(smem_u32(&tmem_base_s), kTmemCols);
     tmem_relinquish();
   }
-  // RoPE tables: cos/sin of pos * base^(-2j/d_axis), computed in double, stored as float2.
+  // RoPE tables (cos / sin in shared memory)
   float4* gcs = reinterpret_cast<float4*>(gb + LY::kTab);   // grouped tables (RT > 0)
   using GR = Groups<(RT > 0 ? RT : 22), (RT > 0 ? RH : 21)>;
-  const int g_count = p.n_frames * GR::GT + p.grid_h * GR::GH + p.grid_w * GR::GW;
-  float2* gns = reinterpret_cast<float2*>(gcs + g_count);
-  if constexpr (RT > 0) {
-    const int offH = p.n_frames * GR::GT, offW = offH + p.grid_h * GR::GH;
-    for (int e = threadIdx.x; e < g_count; e += kThreads) {
-      int pos, g, na;
-      if (e < offH) { pos = e / GR::GT; g = e % GR::GT; na = RT; }
-      else if (e < offW) { pos = (e - offH) / GR::GH; g = (e - offH) % GR::GH; na = RH; }
-      else { pos = (e - offW) / GR::GW; g = (e - offW) % GR::GW; na = GR::RW; }
-      double sn[2] = {0.0, 0.0}, cs[2] = {1.0, 1.0};
-      const bool w_axis = e >= offW;
-#pragma unroll
-      for (int l = 0; l < 2; ++l) {
-        // t, h: record g holds pairs (2g, 2g+1); w: record 0 holds pair 0, record g >= 1
-        // holds pairs (2g-1, 2g)
-        const int jj = w_axis ? (g == 0 ? (l == 0 ? 0 : na) : 2 * g - 1 + l) : 2 * g + l;
-        if (jj < na) {
-          const double turns = static_cast<double>(pos) *
-                               exp2(-(2.0 * jj / (2 * na)) * p.log2_base) * 0.31830988618379067154;
-          sincospi(turns, &sn[l], &cs[l]);
-        }
-      }
-      gcs[e] = make_float4(static_cast<float>(cs[0]), static_cast<float>(cs[1]),
-                           static_cast<float>(sn[0]), static_cast<float>(sn[1]));
-      gns[e] = make_float2(-static_cast<float>(sn[0]), -static_cast<float>(sn[1]));
-    }
-  }
-  // Layout [position][pair j]; 3-D: t (frames), h (grid rows), w (grid columns); 1-D: angle
-  // of the frame offset frame*L_f, then of the in-frame token index.
-  for (int e = threadIdx.x; RT == 0 && e < p.tab_entries; e += kThreads) {
-    int pos, j, da;
-    if (p.rope_mode == 3) {
-      if (e < p.tab_h_off) { pos = e / p.rd[0]; j = e % p.rd[0]; da = 2 * p.rd[0]; }
-      else if (e < p.tab_w_off) { const int f = e - p.tab_h_off; pos = f / p.rd[1]; j = f % p.rd[1]; da = 2 * p.rd[1]; }
-      else { const int f = e - p.tab_w_off; pos = f / p.rd[2]; j = f % p.rd[2]; da = 2 * p.rd[2]; }
-    } else {
-      da = D;
-      if (e < p.tab_h_off) { pos = (e / (D / 2)) * p.L_f; j = e % (D / 2); }
-      else { const int f = e - p.tab_h_off; pos = f / (D / 2); j = f % (D / 2); }
-    }
-    // angle / pi, so that the reduction of the argument is exact (sincospi)
-    const double turns = static_cast<double>(pos) * exp2(-(2.0 * j / da) * p.log2_base) *
-                         0.31830988618379067154;
-    double sn, cs;
-    sincospi(turns, &sn, &cs);
-    tab[e] = make_float2(static_cast<float>(cs), static_cast<float>(sn));
-  }
+  float2* gns = reinterpret_cast<float2*>(
+      gcs + (p.n_frames * GR::GT + p.grid_h * GR::GH + p.grid_w * GR::GW));
+  build_rope_tables<D, RT, RH>(gb + LY::kTab, p, threadIdx.x, kThreads);
   __syncthreads();
   if (warp == 0) {
     // compact the live tiles, 32 at a time, keeping their order
@@ -396,8 +440,19 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
       const uint32_t live = __ballot_sync(0xffffffffu, f & 1);
       if (f & 1)
         tile_list[base + __popc(live & ((1u << lane) - 1u))] =
-            static_cast<uint16_t>(n | ((f & 2) ? 0x8000 : 0));
+            static_cast<uint16_t>(n | ((f & 2) ? (kTileMask | kTileVfix) : 0));
       base += __popc(live);
+    }
+    if (kFused) {
+      // the current block's tiles after the sink tiles; tile i is stored by CTA i mod gridDim.x
+      for (int i = lane; i < p.n_cur_tiles; i += 32) {
+        uint16_t e = static_cast<uint16_t>(i) | kTileNew;
+        if ((i + 1) * BN > p.L_blk) e |= kTileMask;
+        if (i % static_cast<int>(gridDim.x) == static_cast<int>(blockIdx.x))
+          e |= kTileStore | kTileVfix;
+        tile_list[base + i] = e;
+      }
+      base += p.n_cur_tiles;
     }
     if (lane == 0) n_live_s = base;
   }
@@ -421,20 +476,23 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
                       q0 + qt * BM);
       int j = 0, last_k = -1, last_v = -1;               // last iterations whose loads went out
       for (; j < n_live; ++j) {
-        const int n = tile_list[j] & 0x7fff;
+        const uint16_t te = tile_list[j];
+        const int n = te & kTileIdx;
+        const bool cur = kFused && (te & kTileNew);    // [tokens][H][d] map: (d, head, token)
+        const int c1 = cur ? h : n * BN, c2 = cur ? n * BN : h;
         const int st = j & 1;
         const uint32_t par = ((j >> 1) - 1) & 1;
         if (j >= 2 && !mbar_wait(bar(B_KEMPTY + st), par, &ab, deadline, p.status)) break;
         mbar_arrive_expect_tx(bar(B_KFULL + st), LY::kTileBytes);
         for (int pp = 0; pp < D / 64; ++pp)
-          tma_load_3d(sK + st * LY::kTileBytes + pp * 16384, &tm_k, bar(B_KFULL + st), pp * 64,
-                      n * BN, h);
+          tma_load_3d(sK + st * LY::kTileBytes + pp * 16384, cur ? &tm_kn : &tm_k,
+                      bar(B_KFULL + st), pp * 64, c1, c2);
         last_k = j;
         if (j >= 2 && !mbar_wait(bar(B_VEMPTY + st), par, &ab, deadline, p.status)) break;
         mbar_arrive_expect_tx(bar(B_VFULL + st), LY::kTileBytes);
         for (int pp = 0; pp < D / 64; ++pp)
-          tma_load_3d(sV + st * LY::kTileBytes + pp * 16384, &tm_v, bar(B_VFULL + st), pp * 64,
-                      n * BN, h);
+          tma_load_3d(sV + st * LY::kTileBytes + pp * 16384, cur ? &tm_vn : &tm_v,
+                      bar(B_VFULL + st), pp * 64, c1, c2);
         last_v = j;
       }
       if (ab.flag) {     // let copies in flight land before the CTA's shared memory goes away
@@ -478,7 +536,7 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
       int j = 0;
       bool prev_partial = false;
       for (; ok && j < n_live; ++j) {
-        const bool partial = tile_list[j] >> 15;
+        const bool partial = tile_list[j] & kTileVfix;    // V touched by the rotation warps
         const int st = j & 1;
         // P0(j-1).V(j-1) does not need K(j): issue it before waiting for the rotation
         if (j >= 1 && !pv_mma(0, j - 1, prev_partial)) { ok = false; break; }
@@ -531,49 +589,90 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
       mbar_arrive(bar(B_QREADY));
       // position of this thread's key row, advanced incrementally from tile to tile
       int cur = -2 * BN, s_cur = 0, frame = 0, y = 0, x = 0;   // no previous row yet
+      int n_stored = 0;                                         // raw K tiles stored so far
       for (int j = 0; j < n_live; ++j) {
         const uint16_t te = tile_list[j];
-        const int n = te & 0x7fff;
-        const bool partial = te >> 15;
+        const int n = te & kTileIdx;
         const int st = j & 1;
+        const uint32_t kt = sK + st * LY::kTileBytes;
         if (!mbar_wait(bar(B_KFULL + st), (j >> 1) & 1, &ab, deadline, p.status)) break;
-        const int row = n * BN + rt;
         bool empty = false;
-        if (row < p.T) {
-          if (row == cur + BN && row < p.slot_start[s_cur + 1]) {
-            x += p.step_x;                       // one tile further in the same slot
-            y += p.step_y;
-            if (x >= p.grid_w) { x -= p.grid_w; ++y; }
-            while (y >= p.grid_h) { y -= p.grid_h; ++frame; }
-          } else {
-            s_cur = slot_of(row, p);
-            const int u = row - p.slot_start[s_cur];
-            const int tok = u % p.L_f;
-            frame = p.slot_frame[s_cur] + u / p.L_f;
-            y = tok / p.grid_w;
-            x = tok - y * p.grid_w;
+        if (kFused && (te & kTileNew)) {
+          // the current block: store the raw tile into its ring slot (one CTA per tile), then
+          // rotate it at the current block's positions
+          if (te & kTileStore) {
+            if (rt == 0) {
+              for (int pp = 0; pp < D / 64; ++pp)
+                tma_store_3d(&tm_ks, kt + pp * 16384, pp * 64, n * BN, h);
+              bulk_commit();
+              bulk_wait_read_all();
+              mbar_arrive(bar(B_KSTORED));
+            }
+            if (!mbar_wait(bar(B_KSTORED), n_stored & 1, &ab, deadline, p.status)) break;
+            ++n_stored;
           }
-          cur = row;
-          empty = !((vm >> s_cur) & 1u);
-          if constexpr (RT > 0)
-            rotate_row_grouped<RT, RH>(sK + st * LY::kTileBytes, rt, frame, y, x, empty,
-                                       smem_u32(gcs), smem_u32(gns), p);
-          else
-            rotate_row<D, RT, RH>(gb + LY::kK + st * LY::kTileBytes, rt, frame, y, x, empty, tab,
-                                  p);
+          const int ti = n * BN + rt;
+          if (ti < p.L_blk) {
+            const int tok = ti % p.L_f;
+            if constexpr (RT > 0)
+              rotate_row_grouped<RT, RH>(kt, rt, p.q_frame + ti / p.L_f, tok / p.grid_w,
+                                         tok % p.grid_w, false, smem_u32(gcs), smem_u32(gns), p);
+            else
+              rotate_row<D, RT, RH>(gb + LY::kK + st * LY::kTileBytes, rt, p.q_frame + ti / p.L_f,
+                                    tok / p.grid_w, tok % p.grid_w, false, tab, p);
+          }
+        } else if (kFused) {
+          // a tile of the rotated copy: nothing to rotate; find empty-slot rows for V
+          const int row = n * BN + rt;
+          if ((te & kTileVfix) && row < p.T) empty = !((vm >> slot_of(row, p)) & 1u);
+        } else {
+          const int row = n * BN + rt;
+          if (row < p.T) {
+            if (row == cur + BN && row < p.slot_start[s_cur + 1]) {
+              x += p.step_x;                       // one tile further in the same slot
+              y += p.step_y;
+              if (x >= p.grid_w) { x -= p.grid_w; ++y; }
+              while (y >= p.grid_h) { y -= p.grid_h; ++frame; }
+            } else {
+              s_cur = slot_of(row, p);
+              const int u = row - p.slot_start[s_cur];
+              const int tok = u % p.L_f;
+              frame = p.slot_frame[s_cur] + u / p.L_f;
+              y = tok / p.grid_w;
+              x = tok - y * p.grid_w;
+            }
+            cur = row;
+            empty = !((vm >> s_cur) & 1u);
+            if constexpr (RT > 0)
+              rotate_row_grouped<RT, RH>(kt, rt, frame, y, x, empty, smem_u32(gcs),
+                                         smem_u32(gns), p);
+            else
+              rotate_row<D, RT, RH>(gb + LY::kK + st * LY::kTileBytes, rt, frame, y, x, empty,
+                                    tab, p);
+          }
         }
         fence_proxy_async_smem();
         mbar_arrive(bar(B_KREADY + st));
-        if (partial) {
+        if (te & kTileVfix) {
           // boundary tile: empty-slot rows of V may hold anything; P is 0 there, but 0 * NaN
-          // is not, so zero them before the P.V MMA reads the tile
+          // is not, so zero them before the P.V MMA reads the tile.  A current-block tile this
+          // CTA stores: its raw V goes to the ring slot before the P.V MMA may release it.
           if (!mbar_wait(bar(B_VFULL + st), (j >> 1) & 1, &ab, deadline, p.status)) break;
-          if (empty) rotate_row<D, RT, RH>(gb + LY::kV + st * LY::kTileBytes, rt, 0, 0, 0, true,
-                                           tab, p);
+          if (kFused && (te & kTileStore)) {
+            if (rt == 0) {
+              for (int pp = 0; pp < D / 64; ++pp)
+                tma_store_3d(&tm_vs, sV + st * LY::kTileBytes + pp * 16384, pp * 64, n * BN, h);
+              bulk_commit();
+              bulk_wait_read_all();
+            }
+          } else if (empty) {
+            rotate_row<D, RT, RH>(gb + LY::kV + st * LY::kTileBytes, rt, 0, 0, 0, true, tab, p);
+          }
           fence_proxy_async_smem();
           mbar_arrive(bar(B_VFIX + st));
         }
       }
+      if (kFused && rt == 0) bulk_wait_all();    // the ring-slot stores complete before exit
     }
   } else {
     // ------------------------------------------------------------------ softmax (warps 0-7)
@@ -589,7 +688,7 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
     bool ok = true;
     for (; j < n_live; ++j) {
       const uint16_t te = tile_list[j];
-      const int n = te & 0x7fff;
+      const int n = te & kTileIdx;
       ok = mbar_wait(bar(B_SFULL + qt), j & 1, &ab, deadline, p.status);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }   // tcgen05.ld is warp-collective
       tc_fence_after();
@@ -599,13 +698,18 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
       tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
       tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
       tmem_wait_ld();
-      if (te >> 15) {
-        // columns of empty slots and past the end of the cache: 4 mask words, built per slot
+      if (te & kTileMask) {
+        // columns of empty slots and past the end of the cache (or, for the current block's
+        // last tile, past its last token): 4 mask words, built per slot
         const int lo = n * BN;
         uint32_t mw[4] = {~0u, ~0u, ~0u, ~0u};
-        for (int s2 = 0; s2 <= p.n_slots; ++s2) {
+        const bool cur_tile = kFused && (te & kTileNew);
+        for (int s2 = cur_tile ? p.n_slots : 0; s2 <= p.n_slots; ++s2) {
           int a, e;
-          if (s2 < p.n_slots) {
+          if (cur_tile) {
+            a = p.L_blk - lo;
+            e = BN;
+          } else if (s2 < p.n_slots) {
             if ((vm >> s2) & 1u) continue;
             a = p.slot_start[s2] - lo;
             e = p.slot_start[s2 + 1] - lo;
@@ -730,6 +834,128 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
   }
 }
 
+// ---------------------------------------------------------------------------- rotation pass
+// prsink_rotate_sinks: the raw keys of the slots in the rotation mask rotated at this block's
+// positions into k_rot (same [H][T][d] layout), with the attention kernel's own rotation code,
+// so that the fused attention reads keys bitwise equal to the ones it would rotate itself.
+// Work item = (head, key tile of 128 rows); a CTA streams its items through two shared-memory
+// stages: TMA load of the raw tile, one row per thread rotated in place, TMA store.  Rows of
+// other slots that share a boundary tile are rotated and stored too: their rotated copies are
+// either rewritten identically (slots whose positions are fixed) or never read.
+constexpr int kRotThreads = 128;
+
+template <int D, int RT, int RH>
+__global__ void __launch_bounds__(kRotThreads)
+prsink_rotate_kernel(const __grid_constant__ CUtensorMap tm_src,
+                     const __grid_constant__ CUtensorMap tm_dst, const Params p) {
+  using LY = Layout<D>;
+  extern __shared__ uint8_t dsmem[];
+  __shared__ __align__(8) uint64_t full[2];
+  __shared__ AbortState ab;
+  __shared__ unsigned mask_s;
+  __shared__ uint16_t tile_list[kMaxTiles];
+  __shared__ int n_live_s;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rt = threadIdx.x;
+  const uint32_t raw = smem_u32(dsmem);
+  const uint32_t sb = (raw + 1023u) & ~1023u;
+  uint8_t* gb = dsmem + (sb - raw);
+  constexpr int kTabOff = 2 * LY::kTileBytes;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&full[0]), 1);
+    mbar_init(smem_u32(&full[1]), 1);
+    ab.flag = 0;
+    unsigned m = p.rot_mask & p.valid_mask;
+    if (p.cur_slot >= 0) m &= ~(1u << p.cur_slot);
+    if ((p.dyn_src && *p.dyn_src < 0) || (p.rot_dyn_flag && *p.rot_dyn_flag == 0))
+      m &= ~(1u << PRSINK_SLOT_DYNAMIC);
+    mask_s = m;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  float4* gcs = reinterpret_cast<float4*>(gb + kTabOff);
+  using GR = Groups<(RT > 0 ? RT : 22), (RT > 0 ? RH : 21)>;
+  float2* gns = reinterpret_cast<float2*>(
+      gcs + (p.n_frames * GR::GT + p.grid_h * GR::GH + p.grid_w * GR::GW));
+  float2* tab = reinterpret_cast<float2*>(gb + kTabOff);
+  build_rope_tables<D, RT, RH>(gb + kTabOff, p, threadIdx.x, kRotThreads);
+  if (warp == 0) {
+    const int n_tiles = (p.T + BN - 1) / BN;
+    int base = 0;
+    for (int n0 = 0; n0 < n_tiles; n0 += 32) {
+      const int n = n0 + lane;
+      const bool live = n < n_tiles && tile_live(n, mask_s, p);
+      const uint32_t bal = __ballot_sync(0xffffffffu, live);
+      if (live) tile_list[base + __popc(bal & ((1u << lane) - 1u))] = static_cast<uint16_t>(n);
+      base += __popc(bal);
+    }
+    if (lane == 0) n_live_s = base;
+  }
+  __syncthreads();
+  const int n_live = n_live_s;
+  const int total = n_live * p.H;
+  const uint64_t deadline = globaltimer() + p.timeout_ns;
+  auto item = [&](int w, int& n, int& h) { h = w / n_live; n = tile_list[w - h * n_live]; };
+  auto load = [&](int w, int st) {
+    int n, h;
+    item(w, n, h);
+    const uint32_t bar = smem_u32(&full[st]);
+    mbar_arrive_expect_tx(bar, LY::kTileBytes);
+    for (int pp = 0; pp < D / 64; ++pp)
+      tma_load_3d(sb + st * LY::kTileBytes + pp * 16384, &tm_src, bar, pp * 64, n * BN, h);
+  };
+  int i = 0, last_load = -1;
+  if (threadIdx.x == 0 && static_cast<int>(blockIdx.x) < total) {
+    prefetch_tmap(&tm_src);
+    prefetch_tmap(&tm_dst);
+    load(blockIdx.x, 0);
+    last_load = 0;
+  }
+  for (int w = blockIdx.x; w < total; w += gridDim.x, ++i) {
+    const int st = i & 1;
+    const int wn = w + gridDim.x;
+    if (threadIdx.x == 0 && wn < total) {
+      bulk_wait_read_all();             // the store of item i-1 has read stage st^1
+      load(wn, st ^ 1);
+      last_load = i + 1;
+    }
+    // every thread takes the same decision (a wait that gave up in one thread ends the loop
+    // for all, so no thread is left behind at the barrier below)
+    if (!__syncthreads_and(mbar_wait(smem_u32(&full[st]), (i >> 1) & 1, &ab, deadline,
+                                     p.status)))
+      break;
+    int n, h;
+    item(w, n, h);
+    const int row = n * BN + rt;
+    if (row < p.T) {
+      const int s = slot_of(row, p);
+      const int u = row - p.slot_start[s];
+      const int tok = u % p.L_f;
+      const int frame = p.slot_frame[s] + u / p.L_f;
+      if constexpr (RT > 0)
+        rotate_row_grouped<RT, RH>(sb + st * LY::kTileBytes, rt, frame, tok / p.grid_w,
+                                   tok % p.grid_w, false, smem_u32(gcs), smem_u32(gns), p);
+      else
+        rotate_row<D, RT, RH>(gb + st * LY::kTileBytes, rt, frame, tok / p.grid_w,
+                              tok % p.grid_w, false, tab, p);
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      for (int pp = 0; pp < D / 64; ++pp)
+        tma_store_3d(&tm_dst, sb + st * LY::kTileBytes + pp * 16384, pp * 64, n * BN, h);
+      bulk_commit();
+    }
+  }
+  if (threadIdx.x == 0) {
+    if (ab.flag) {                      // let loads in flight land before shared memory goes
+      for (int k = last_load - 1; k <= last_load; ++k)
+        if (k >= i) drain_wait(smem_u32(&full[k & 1]), (k >> 1) & 1, 100000000ull);
+    }
+    bulk_wait_all();
+  }
+}
+
 // ---------------------------------------------------------------------------- host side
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -772,67 +998,114 @@ static int make_map(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, 
   return PRSINK_OK;
 }
 
-template <int D, int RT, int RH>
-static int launch(const prsink_layout* L, const Geometry& g, const void* q, const void* k,
-                  const void* v, Params& p, cudaStream_t st) {
-  CUtensorMap mq, mk, mv;
-  int rc = make_map(&mq, q, D, L->n_heads, g.L_blk, 2ull * D, 2ull * D * L->n_heads, 1, BM);
-  if (!rc) rc = make_map(&mk, k, D, g.T, L->n_heads, 2ull * D, 2ull * D * g.T, BN, 1);
-  if (!rc) rc = make_map(&mv, v, D, g.T, L->n_heads, 2ull * D, 2ull * D * g.T, BN, 1);
-  if (rc) return rc;
+// Device buffers of one call: q, the key / value sources of the slot-indexed tiles (raw caches,
+// or k_rot and v_cache in the fused form), and for the fused form k_new, v_new and the caches
+// whose current ring slot receives the raw block.
+struct Buffers {
+  const void* q;
+  const void* k;
+  const void* v;
+  const void* k_new;
+  const void* v_new;
+  void* k_cache;
+  void* v_cache;
+};
+
+static int table_bytes(const prsink_layout* L, const Params& p, bool grouped) {
   using GR = Groups<22, 21>;
-  const int tab_bytes = RT > 0 ? (p.n_frames * GR::GT + L->grid_h * GR::GH + L->grid_w * GR::GW) * 24
-                               : p.tab_entries * 8;
-  if (tab_bytes > kTableMaxBytes) {
-    set_error("prsink_attention: RoPE tables need %d bytes of shared memory (max %d)", tab_bytes,
-              kTableMaxBytes);
-    return PRSINK_ERR_UNSUPPORTED;
-  }
-  int smem = Layout<D>::kTab + tab_bytes + 1024;
-  if (smem < 120 * 1024) smem = 120 * 1024;     // one CTA per SM (it holds all 512 TMEM columns)
-  static int attr_bytes[64] = {0};      // largest size already allowed, per device
+  return grouped ? (p.n_frames * GR::GT + L->grid_h * GR::GH + L->grid_w * GR::GW) * 24
+                 : p.tab_entries * 8;
+}
+
+// Allow `smem` bytes of dynamic shared memory for `fn` (once per size and device).
+template <typename F>
+static int allow_smem(F fn, int smem, int (&allowed)[64], const char* what) {
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) dev = 0;
-  if (attr_bytes[dev] < smem) {
-    if (cudaFuncSetAttribute(prsink_attention_kernel<D, RT, RH>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-      return check_launch("prsink_attention: shared memory attribute");
-    attr_bytes[dev] = smem;
+  if (allowed[dev] < smem) {
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+        cudaSuccess)
+      return check_launch(what);
+    allowed[dev] = smem;
   }
-  dim3 grid((g.L_blk + NQ * BM - 1) / (NQ * BM), L->n_heads);
-  prsink_attention_kernel<D, RT, RH><<<grid, kThreads, smem, st>>>(mq, mk, mv, p);
-  count_launch();
-  return check_launch("prsink_attention");
+  return PRSINK_OK;
 }
 
-}  // namespace attn
-}  // namespace prsink
-
-using namespace prsink;
-
-extern "C" int prsink_attention(const prsink_layout* layout, const void* q, const void* k_cache,
-                                const void* v_cache, void* out, float* lse,
-                                const long long* dyn_src, void* stream) {
-  using namespace prsink::attn;
-  Geometry g;
-  int rc = geometry(layout, &g);
-  if (rc) return rc;
-  if (!q || !k_cache || !v_cache || !out) {
-    set_error("prsink_attention: null pointer");
-    return PRSINK_ERR_ARG;
+template <int D, int RT, int RH, bool kFused>
+static int launch(const prsink_layout* L, const Geometry& g, const Buffers& b, Params& p,
+                  cudaStream_t st) {
+  const char* what = kFused ? "prsink_attention_fused" : "prsink_attention";
+  const uint64_t H = L->n_heads;
+  CUtensorMap mq, mk, mv, mkn, mvn, mks, mvs;
+  int rc = make_map(&mq, b.q, D, H, g.L_blk, 2ull * D, 2ull * D * H, 1, BM);
+  if (!rc) rc = make_map(&mk, b.k, D, g.T, H, 2ull * D, 2ull * D * g.T, BN, 1);
+  if (!rc) rc = make_map(&mv, b.v, D, g.T, H, 2ull * D, 2ull * D * g.T, BN, 1);
+  if (kFused) {
+    // current block: token-major k_new / v_new; raw store: the ring slot's rows of the caches
+    const uint64_t off = 2ull * D * static_cast<uint64_t>(g.slot_start[p.cur_slot]);
+    if (!rc) rc = make_map(&mkn, b.k_new, D, H, g.L_blk, 2ull * D, 2ull * D * H, 1, BN);
+    if (!rc) rc = make_map(&mvn, b.v_new, D, H, g.L_blk, 2ull * D, 2ull * D * H, 1, BN);
+    if (!rc) rc = make_map(&mks, static_cast<char*>(b.k_cache) + off, D, g.L_blk, H, 2ull * D,
+                           2ull * D * g.T, BN, 1);
+    if (!rc) rc = make_map(&mvs, static_cast<char*>(b.v_cache) + off, D, g.L_blk, H, 2ull * D,
+                           2ull * D * g.T, BN, 1);
+  } else {
+    mkn = mvn = mks = mvs = mk;                 // unused
   }
-  const int D = layout->head_dim;
-  if (D != 64 && D != 128) {
-    set_error("prsink_attention: head_dim %d not supported (64 or 128)", D);
+  if (rc) return rc;
+  const int tab = table_bytes(L, p, RT > 0);
+  if (tab > kTableMaxBytes) {
+    set_error("%s: RoPE tables need %d bytes of shared memory (max %d)", what, tab,
+              kTableMaxBytes);
     return PRSINK_ERR_UNSUPPORTED;
   }
-  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
-      (lse && (reinterpret_cast<uintptr_t>(lse) & 3u))) {
-    set_error("prsink_attention: q, k_cache, v_cache, out must be 16-byte aligned");
-    return PRSINK_ERR_ALIGN;
+  int smem = Layout<D>::kTab + tab + 1024;
+  if (smem < 120 * 1024) smem = 120 * 1024;     // one CTA per SM (it holds all 512 TMEM columns)
+  static int allowed[64] = {0};
+  rc = allow_smem(prsink_attention_kernel<D, RT, RH, kFused>, smem, allowed, what);
+  if (rc) return rc;
+  dim3 grid((g.L_blk + NQ * BM - 1) / (NQ * BM), L->n_heads);
+  prsink_attention_kernel<D, RT, RH, kFused><<<grid, kThreads, smem, st>>>(mq, mk, mv, mkn, mvn,
+                                                                          mks, mvs, p);
+  count_launch();
+  return check_launch(what);
+}
+
+template <int D, int RT, int RH>
+static int launch_rotate(const prsink_layout* L, const Geometry& g, const void* k_cache,
+                         void* k_rot, Params& p, cudaStream_t st) {
+  const uint64_t H = L->n_heads;
+  CUtensorMap ms, md;
+  int rc = make_map(&ms, k_cache, D, g.T, H, 2ull * D, 2ull * D * g.T, BN, 1);
+  if (!rc) rc = make_map(&md, k_rot, D, g.T, H, 2ull * D, 2ull * D * g.T, BN, 1);
+  if (rc) return rc;
+  const int tab = table_bytes(L, p, RT > 0);
+  if (tab > kTableMaxBytes) {
+    set_error("prsink_rotate_sinks: RoPE tables need %d bytes of shared memory (max %d)", tab,
+              kTableMaxBytes);
+    return PRSINK_ERR_UNSUPPORTED;
   }
-  Params p{};
+  const int smem = 2 * Layout<D>::kTileBytes + tab + 1024;
+  static int allowed[64] = {0};
+  rc = allow_smem(prsink_rotate_kernel<D, RT, RH>, smem, allowed, "prsink_rotate_sinks");
+  if (rc) return rc;
+  int n_sm = 148, dev = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
+  // work items: every (head, key tile); two CTAs per SM stream them
+  const long long items = static_cast<long long>(H) * ((g.T + BN - 1) / BN);
+  const int grid = static_cast<int>(items < 2ll * n_sm ? items : 2ll * n_sm);
+  prsink_rotate_kernel<D, RT, RH><<<grid, kRotThreads, smem, st>>>(ms, md, p);
+  count_launch();
+  return check_launch("prsink_rotate_sinks");
+}
+
+// Parameters shared by every kernel of this file, from the layout (validated by the caller).
+static int fill_params(const prsink_layout* layout, const Geometry& g, Params& p,
+                       const char* what) {
+  const int D = layout->head_dim;
+  p = Params{};
   p.H = layout->n_heads;
   p.L_blk = static_cast<int>(g.L_blk);
   p.T = static_cast<int>(g.T);
@@ -875,26 +1148,136 @@ extern "C" int prsink_attention(const prsink_layout* layout, const void* q, cons
   p.step_y = BN / layout->grid_w;
   p.step_x = BN % layout->grid_w;
   if ((g.T + BN - 1) / BN > kMaxTiles) {
-    set_error("prsink_attention: %lld keys exceed the %d-tile limit", g.T, kMaxTiles);
+    set_error("%s: %lld keys exceed the %d-tile limit", what, g.T, kMaxTiles);
     return PRSINK_ERR_UNSUPPORTED;
   }
   if (p.tab_entries * 8 > kTableMaxBytes) {
-    set_error("prsink_attention: RoPE tables need %d bytes of shared memory (max %d)",
+    set_error("%s: RoPE tables need %d bytes of shared memory (max %d)", what,
               p.tab_entries * 8, kTableMaxBytes);
     return PRSINK_ERR_UNSUPPORTED;
   }
   p.log2_base = std::log2(static_cast<double>(layout->rope_base));
   p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
+  p.status = status_word_ptr();
+  p.timeout_ns = 2000000000ull;
+  p.cur_slot = -1;
+  if (!p.status) return PRSINK_ERR_LAUNCH;
+  return PRSINK_OK;
+}
+
+static bool grouped_split(const prsink_layout* L, const Params& p) {
+  return L->head_dim == 128 && p.rope_mode == 3 && p.rd[0] == 22 && p.rd[1] == 21;
+}
+
+template <bool kFused>
+static int dispatch(const prsink_layout* L, const Geometry& g, const Buffers& b, Params& p,
+                    cudaStream_t st) {
+  if (grouped_split(L, p)) return launch<128, 22, 21, kFused>(L, g, b, p, st);   // 44/42/42
+  return L->head_dim == 128 ? launch<128, 0, 0, kFused>(L, g, b, p, st)
+                            : launch<64, 0, 0, kFused>(L, g, b, p, st);
+}
+
+// Common checks of the attention entry points.
+static int check_attention_args(const prsink_layout* layout, Geometry* g, const char* what,
+                                std::initializer_list<const void*> bufs, const float* lse) {
+  int rc = geometry(layout, g);
+  if (rc) return rc;
+  for (const void* ptr : bufs)
+    if (!ptr) {
+      set_error("%s: null pointer", what);
+      return PRSINK_ERR_ARG;
+    }
+  const int D = layout->head_dim;
+  if (D != 64 && D != 128) {
+    set_error("%s: head_dim %d not supported (64 or 128)", what, D);
+    return PRSINK_ERR_UNSUPPORTED;
+  }
+  for (const void* ptr : bufs)
+    if (!aligned16(ptr)) {
+      set_error("%s: every K/V/Q/out buffer must be 16-byte aligned", what);
+      return PRSINK_ERR_ALIGN;
+    }
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) {
+    set_error("%s: lse must be 4-byte aligned", what);
+    return PRSINK_ERR_ALIGN;
+  }
+  return PRSINK_OK;
+}
+
+}  // namespace attn
+}  // namespace prsink
+
+using namespace prsink;
+
+extern "C" int prsink_attention(const prsink_layout* layout, const void* q, const void* k_cache,
+                                const void* v_cache, void* out, float* lse,
+                                const long long* dyn_src, void* stream) {
+  using namespace prsink::attn;
+  Geometry g;
+  int rc = check_attention_args(layout, &g, "prsink_attention", {q, k_cache, v_cache, out}, lse);
+  if (rc) return rc;
+  Params p;
+  rc = fill_params(layout, g, p, "prsink_attention");
+  if (rc) return rc;
   p.out = static_cast<__nv_bfloat16*>(out);
   p.lse = lse;
   p.dyn_src = dyn_src;
-  p.status = status_word_ptr();
-  p.timeout_ns = 2000000000ull;
-  if (!p.status) return PRSINK_ERR_LAUNCH;
   if (g.L_blk == 0) return PRSINK_OK;
+  const Buffers b{q, k_cache, v_cache, nullptr, nullptr, nullptr, nullptr};
+  return dispatch<false>(layout, g, b, p, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int prsink_attention_fused(const prsink_layout* layout, const void* q,
+                                      const void* k_new, const void* v_new, const void* k_rot,
+                                      void* k_cache, void* v_cache, void* out, float* lse,
+                                      const long long* dyn_src, void* stream) {
+  using namespace prsink::attn;
+  Geometry g;
+  int rc = check_attention_args(layout, &g, "prsink_attention_fused",
+                                {q, k_new, v_new, k_rot, k_cache, v_cache, out}, lse);
+  if (rc) return rc;
+  if (k_rot == k_cache) {
+    set_error("prsink_attention_fused: k_rot must be a buffer of its own");
+    return PRSINK_ERR_ARG;
+  }
+  Params p;
+  rc = fill_params(layout, g, p, "prsink_attention_fused");
+  if (rc) return rc;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.dyn_src = dyn_src;
+  p.cur_slot = PRSINK_SLOT_RING0 + static_cast<int>(layout->block_index % layout->ring_slots);
+  p.n_cur_tiles = static_cast<int>((g.L_blk + BN - 1) / BN);
+  if ((g.T + BN - 1) / BN + p.n_cur_tiles > kMaxTiles) {
+    set_error("prsink_attention_fused: %lld keys exceed the tile limit", g.T);
+    return PRSINK_ERR_UNSUPPORTED;
+  }
+  if (g.L_blk == 0) return PRSINK_OK;
+  const Buffers b{q, k_rot, v_cache, k_new, v_new, k_cache, v_cache};
+  return dispatch<true>(layout, g, b, p, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int prsink_rotate_sinks(const prsink_layout* layout, const void* k_cache,
+                                   void* k_rot, unsigned slot_mask, const int* dyn_flag,
+                                   const long long* dyn_src, void* stream) {
+  using namespace prsink::attn;
+  Geometry g;
+  int rc = check_attention_args(layout, &g, "prsink_rotate_sinks", {k_cache, k_rot}, nullptr);
+  if (rc) return rc;
+  if (k_rot == k_cache) {
+    set_error("prsink_rotate_sinks: k_rot must be a buffer of its own");
+    return PRSINK_ERR_ARG;
+  }
+  Params p;
+  rc = fill_params(layout, g, p, "prsink_rotate_sinks");
+  if (rc) return rc;
+  p.cur_slot = PRSINK_SLOT_RING0 + static_cast<int>(layout->block_index % layout->ring_slots);
+  p.rot_mask = slot_mask;
+  p.rot_dyn_flag = dyn_flag;
+  p.dyn_src = dyn_src;
+  if ((slot_mask & p.valid_mask & ~(1u << p.cur_slot)) == 0) return PRSINK_OK;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (D == 128 && p.rope_mode == 3 && p.rd[0] == 22 && p.rd[1] == 21)   // 44/42/42 split
-    return launch<128, 22, 21>(layout, g, q, k_cache, v_cache, p, st);
-  return D == 128 ? launch<128, 0, 0>(layout, g, q, k_cache, v_cache, p, st)
-                  : launch<64, 0, 0>(layout, g, q, k_cache, v_cache, p, st);
+  if (grouped_split(layout, p)) return launch_rotate<128, 22, 21>(layout, g, k_cache, k_rot, p, st);
+  return layout->head_dim == 128 ? launch_rotate<128, 0, 0>(layout, g, k_cache, k_rot, p, st)
+                                 : launch_rotate<64, 0, 0>(layout, g, k_cache, k_rot, p, st);
 }

@@ -45,10 +45,13 @@ class PRSinkStream:
 
     def __init__(self, cfg: dict, n_layers: int, M: int = 5, write_blocks: int = 20,
                  device="cuda", policy: str = "frozen", alpha: float = 0.0, gate: float = 0.0,
-                 min_detected: int = 0):
+                 min_detected: int = 0, fused: bool = False):
         """``policy``, ``alpha``, ``gate``: the bank policy (the pages' frozen bank, or one of
         the variants of ``prsink_bank_update_policy``); ``min_detected`` > 0 makes retrieval
-        fall back to Static Sink + window for blocks with fewer detected frames."""
+        fall back to Static Sink + window for blocks with fewer detected frames.  ``fused``:
+        each layer keeps a rotated copy of its sink keys, refreshed once per block by
+        ``prsink_rotate_sinks``, and every pass is one ``prsink_attention_fused`` launch (the
+        append folded in) instead of an append and a ``prsink_attention`` launch."""
         self.cfg = dict(cfg)
         self.n_layers, self.M, self.write_blocks = int(n_layers), int(M), int(write_blocks)
         self.policy = L.make_policy(policy, write_blocks, alpha, gate)
@@ -72,6 +75,11 @@ class PRSinkStream:
         self.action = torch.zeros(1, dtype=torch.int32, device=dev)
         self.mode = torch.zeros(1, dtype=torch.int32, device=dev)
         self.frame_ok = torch.ones(3, dtype=torch.uint8, device=dev)
+        self.fused = bool(fused)
+        self.k_rot = (torch.zeros((n_layers, H, self.T, d), dtype=bf, device=dev)
+                      if self.fused else None)
+        self._rot_pending = [0] * self.n_layers     # ref / static slots written since rotated
+        self._rot_block = [-1] * self.n_layers      # block of each layer's last rotation pass
         self.b = 0
 
     def reset(self):
@@ -82,6 +90,7 @@ class PRSinkStream:
         self.bank_src.fill_(-1)
         self.bank_count.zero_()
         self.dyn_src.fill_(-1)
+        self._rot_block = [-1] * self.n_layers
         self.b = 0
 
     def layout(self, b: int = None) -> L.Layout:
@@ -95,6 +104,7 @@ class PRSinkStream:
     def set_ref(self, layer: int, k_ref, v_ref, stream=None):
         k, v = self.kv(layer)
         L.prsink_kv_append(self.layout(), k_ref, v_ref, k, v, L.SLOT_REF, stream)
+        self._rot_pending[layer] |= 1 << L.SLOT_REF
 
     def begin_block(self, kp, frame_ok, stream=None):
         """Fingerprint (kp f32 [3][62][3], frame_ok u8 [3], on the device) and retrieval."""
@@ -116,6 +126,22 @@ class PRSinkStream:
         into the static sink), then attend."""
         lay = self.layout()
         k, v = self.kv(layer)
+        if self.fused:
+            if self._rot_block[layer] != self.b:
+                # ring slots move one rank per block; the dynamic slot when retrieval refilled
+                # it; ref and static once after they were written
+                ring = ((1 << self.R) - 1) << L.SLOT_RING0
+                mask = ring | (1 << L.SLOT_DYNAMIC) | self._rot_pending[layer]
+                L.prsink_rotate_sinks(lay, k, self.k_rot[layer], mask, self.copied,
+                                      self.dyn_src, stream)
+                self._rot_pending[layer] = 0
+                self._rot_block[layer] = self.b
+            L.prsink_attention_fused(lay, q, k_new, v_new, self.k_rot[layer], k, v, out, lse,
+                                     self.dyn_src, stream)
+            if clean and self.b == 0:
+                L.prsink_kv_append(lay, k_new, v_new, k, v, L.SLOT_STATIC, stream)
+                self._rot_pending[layer] |= 1 << L.SLOT_STATIC
+            return
         L.prsink_kv_append(lay, k_new, v_new, k, v, L.SLOT_RING0 + self.b % self.R, stream)
         if clean and self.b == 0:
             L.prsink_kv_append(lay, k_new, v_new, k, v, L.SLOT_STATIC, stream)
