@@ -306,6 +306,15 @@ long long prsink_launch_count(void);
  * PRSINK_ERR_TIMEOUT in the status word and returns.  No GPU fault, no hang. */
 int prsink_debug_wait_timeout(long long timeout_ns, void* stream);
 
+/* Self-test of the attention kernel's own abort path.  Arms the next prsink_attention /
+ * prsink_attention_fused / prsink_rotate_sinks call of this host thread (one call only): its
+ * bounded waits give up after `timeout_ns` (clamped to [1e4, 1e9] ns) instead of 2 s, and in an
+ * attention call the MMA issuer withholds the first commit of query tile 0, so that the softmax
+ * wait runs out.  The kernel then raises its abort flag, records PRSINK_ERR_TIMEOUT in the status
+ * word, lets its copies and MMAs in flight complete, frees its tensor memory and writes out = 0,
+ * lse = -inf for the rows it did not finish.  No GPU fault, no hang; the next call is normal. */
+int prsink_debug_attention_stall(long long timeout_ns);
+
 /* Library ABI version (increments on any signature change). */
 int prsink_version(void);
 

@@ -110,6 +110,7 @@ def _load():
                                        vp, vp, vp, vp, i, vp], i),
         "prsink_sync_status": ([vp], i),
         "prsink_debug_wait_timeout": ([ll, vp], i),
+        "prsink_debug_attention_stall": ([ll], i),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -126,7 +127,7 @@ def exported_symbols() -> list:
             "prsink_attention", "prsink_kv_append", "prsink_fingerprint", "prsink_retrieve",
             "prsink_bank_update", "prsink_sync_status", "prsink_debug_wait_timeout",
             "prsink_retrieve_fallback", "prsink_bank_update_policy", "prsink_attention_fused",
-            "prsink_rotate_sinks"]
+            "prsink_rotate_sinks", "prsink_debug_attention_stall"]
 
 
 def _check(rc: int, fn: str):
@@ -332,3 +333,7 @@ def prsink_sync_status(stream=None) -> int:
 def prsink_debug_wait_timeout(timeout_ns: int, stream=None):
     _check(_lib.prsink_debug_wait_timeout(int(timeout_ns), _stream(stream)),
            "prsink_debug_wait_timeout")
+
+
+def prsink_debug_attention_stall(timeout_ns: int):
+    _check(_lib.prsink_debug_attention_stall(int(timeout_ns)), "prsink_debug_attention_stall")

@@ -68,6 +68,7 @@ struct Params {
   // rotation pass (prsink_rotate_sinks): slots whose rows are rotated into k_rot
   unsigned rot_mask;
   const int* rot_dyn_flag;              // dynamic slot rotated only if *flag != 0 (nullable)
+  int debug_stall;                      // self-test: withhold the first S commit of query tile 0
 };
 
 // Entries of the per-CTA tile list: a key tile index and what the roles do with it.
@@ -543,7 +544,9 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
         if (!mbar_wait(bar(B_KREADY + st), (j >> 1) & 1, &ab, deadline, p.status)) { ok = false; break; }
         tc_fence_after();
         s_mma(0, st);
-        umma_commit(bar(B_SFULL + 0));
+        // self-test of the abort path: without this commit the softmax of tile 0 waits until
+        // its deadline, raises the abort flag and every role drains and exits
+        if (!(p.debug_stall && j == 0)) umma_commit(bar(B_SFULL + 0));
         if (j >= 1) {
           if (!pv_mma(1, j - 1, prev_partial)) { ok = false; break; }
           umma_commit(bar(B_VEMPTY + ((j - 1) & 1)));
@@ -1101,6 +1104,9 @@ static int launch_rotate(const prsink_layout* L, const Geometry& g, const void* 
   return check_launch("prsink_rotate_sinks");
 }
 
+// Self-test of the attention kernel's abort path (per host thread, one call).
+static thread_local long long g_debug_stall_ns = 0;
+
 // Parameters shared by every kernel of this file, from the layout (validated by the caller).
 static int fill_params(const prsink_layout* layout, const Geometry& g, Params& p,
                        const char* what) {
@@ -1161,6 +1167,11 @@ static int fill_params(const prsink_layout* layout, const Geometry& g, Params& p
   p.status = status_word_ptr();
   p.timeout_ns = 2000000000ull;
   p.cur_slot = -1;
+  if (g_debug_stall_ns > 0) {           // armed by prsink_debug_attention_stall: one call only
+    p.debug_stall = 1;
+    p.timeout_ns = static_cast<unsigned long long>(g_debug_stall_ns);
+    g_debug_stall_ns = 0;
+  }
   if (!p.status) return PRSINK_ERR_LAUNCH;
   return PRSINK_OK;
 }
@@ -1280,4 +1291,11 @@ extern "C" int prsink_rotate_sinks(const prsink_layout* layout, const void* k_ca
   if (grouped_split(layout, p)) return launch_rotate<128, 22, 21>(layout, g, k_cache, k_rot, p, st);
   return layout->head_dim == 128 ? launch_rotate<128, 0, 0>(layout, g, k_cache, k_rot, p, st)
                                  : launch_rotate<64, 0, 0>(layout, g, k_cache, k_rot, p, st);
+}
+
+extern "C" int prsink_debug_attention_stall(long long timeout_ns) {
+  if (timeout_ns < 10000) timeout_ns = 10000;
+  if (timeout_ns > 1000000000ll) timeout_ns = 1000000000ll;
+  prsink::attn::g_debug_stall_ns = timeout_ns;
+  return PRSINK_OK;
 }

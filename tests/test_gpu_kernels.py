@@ -195,3 +195,26 @@ def test_launch_counter_counts_kernels():
     P.prsink_kv_append(P.make_layout(**cfg), q, q, k, k, 3)
     torch.cuda.synchronize()
     assert P.prsink_launch_count() == n0 + 2
+
+
+def test_attention_abort_path_reports_timeout_and_recovers():
+    """The attention kernel's own abort path: a one-shot self-test makes the MMA issuer withhold
+    one commit, so the softmax wait runs out after 2 ms.  The kernel must record the timeout,
+    drain its copies and MMAs, free its tensor memory and write out = 0, lse = -inf; the next
+    normal call must match the oracle."""
+    need_gpu()
+    from tests._gpu import attention_inputs, check_attention
+    cfg = synth.preset("tiny", block_index=7, valid_mask=0xFF)
+    q, k, v = attention_inputs(cfg, seed=31)
+    lay = P.make_layout(**cfg)
+    out = torch.full((48, 1, 64), 5.0, dtype=torch.bfloat16, device="cuda")
+    lse = torch.zeros((1, 48), dtype=torch.float32, device="cuda")
+    assert P.prsink_sync_status() == P.PRSINK_OK
+    P.prsink_debug_attention_stall(2_000_000)
+    P.prsink_attention(lay, q.cuda(), k.cuda(), v.cuda(), out, lse)
+    assert P.prsink_sync_status() == P.PRSINK_ERR_TIMEOUT
+    assert torch.all(out == 0) and torch.all(torch.isneginf(lse))
+    P.prsink_attention(lay, q.cuda(), k.cuda(), v.cuda(), out, lse)
+    assert P.prsink_sync_status() == P.PRSINK_OK
+    ref, _ = oracle.attention(cfg, f64(q), f64(k), f64(v))
+    check_attention(f64(out), ref, "after the abort")
