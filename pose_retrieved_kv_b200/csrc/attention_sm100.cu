@@ -373,6 +373,7 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
   __shared__ uint8_t tile_flag[kMaxTiles];       // bit 0: holds a valid key, bit 1: boundary
   __shared__ uint16_t tile_list[kMaxTiles];      // live tiles in order (kTile* bits)
   __shared__ int n_live_s;
+  __shared__ int last_k_s, last_v_s;             // last K / V loads issued (for the drain)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t raw = smem_u32(dsmem);
@@ -402,6 +403,7 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
     mbar_init(bar(B_FINAL), 1);
     mbar_init(bar(B_KSTORED), 1);
     ab.flag = 0;
+    last_k_s = last_v_s = -1;
     unsigned vm = p.valid_mask;
     if (p.dyn_src && *p.dyn_src < 0) vm &= ~(1u << PRSINK_SLOT_DYNAMIC);
     if (kFused) vm &= ~(1u << p.cur_slot);        // its keys come from k_new instead
@@ -496,13 +498,8 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
                       bar(B_VFULL + st), pp * 64, c1, c2);
         last_v = j;
       }
-      if (ab.flag) {     // let copies in flight land before the CTA's shared memory goes away
-        drain_wait(bar(B_QFULL), 0, 100000000ull);
-        for (int i = last_k - 1; i <= last_k; ++i)
-          if (i >= 0) drain_wait(bar(B_KFULL + (i & 1)), (i >> 1) & 1, 100000000ull);
-        for (int i = last_v - 1; i <= last_v; ++i)
-          if (i >= 0) drain_wait(bar(B_VFULL + (i & 1)), (i >> 1) & 1, 100000000ull);
-      }
+      last_k_s = last_k;
+      last_v_s = last_v;
     } else if (warp == kMmaWarp && lane == 0) {
       // ---------------------------------------------------------------- MMA issuer
       bool ok = mbar_wait(bar(B_QREADY), 0, &ab, deadline, p.status);
@@ -564,10 +561,6 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
             umma_commit(bar(B_ODONE + 1));
           }
         }
-      }
-      if (ab.flag) {     // wait for every MMA issued so far before TMEM is released
-        umma_commit(bar(B_FINAL));
-        drain_wait(bar(B_FINAL), 0, 100000000ull);
       }
     }
   } else if (warp >= kRotWarp0) {
@@ -831,6 +824,24 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
 
   tc_fence_before();
   __syncthreads();
+  // Every role has left its loop, so the abort flag is final here.  After an abort, copies and
+  // MMAs may still be in flight: let them complete before the CTA's shared and tensor memory
+  // are released (bounded waits; an abort raised late by one role is seen by all).
+  if (ab.flag) {
+    if (warp == kProducerWarp && lane == 0) {
+      drain_wait(bar(B_QFULL), 0, 100000000ull);
+      for (int i = last_k_s - 1; i <= last_k_s; ++i)
+        if (i >= 0) drain_wait(bar(B_KFULL + (i & 1)), (i >> 1) & 1, 100000000ull);
+      for (int i = last_v_s - 1; i <= last_v_s; ++i)
+        if (i >= 0) drain_wait(bar(B_VFULL + (i & 1)), (i >> 1) & 1, 100000000ull);
+    }
+    if (warp == kMmaWarp && lane == 0) {       // the thread that issued every MMA
+      umma_commit(bar(B_FINAL));
+      drain_wait(bar(B_FINAL), 0, 100000000ull);
+    }
+    tc_fence_before();
+    __syncthreads();
+  }
   if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);

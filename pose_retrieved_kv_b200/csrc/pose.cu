@@ -218,22 +218,18 @@ bank_update_kernel(float* __restrict__ bank_phi, long long* __restrict__ bank_sr
     float* e = bank_phi + static_cast<size_t>(a) * PRSINK_FP_DIM;
     const double w_new = static_cast<double>(pol.alpha);
     const double w_old = static_cast<double>(1.0f - pol.alpha);   // the float32 weight
-    double t[(PRSINK_FP_DIM + 1023) / 1024];
-    double s = 0.0;
-    int k = 0;
-    for (int i = threadIdx.x; i < PRSINK_FP_DIM; i += blockDim.x, ++k) {
-      t[k] = w_old * static_cast<double>(e[i]) + w_new * static_cast<double>(q[i]);
-      s += t[k] * t[k];
-    }
-    s = warp_sum(s);
+    // one element per thread (the kernel runs with 1024 >= 558 threads)
+    const int i = threadIdx.x;
+    const double t = i < PRSINK_FP_DIM
+                         ? w_old * static_cast<double>(e[i]) + w_new * static_cast<double>(q[i])
+                         : 0.0;
+    double s = warp_sum(t * t);
     if (lane == 0) part[warp] = s;
     __syncthreads();
     double n2 = 0.0;
     for (int w = 0; w < nw; ++w) n2 += part[w];
     const double inv = n2 > 0.0 ? 1.0 / sqrt(n2) : 1.0;
-    k = 0;
-    for (int i = threadIdx.x; i < PRSINK_FP_DIM; i += blockDim.x, ++k)
-      e[i] = static_cast<float>(t[k] * inv);
+    if (i < PRSINK_FP_DIM) e[i] = static_cast<float>(t * inv);
   }
 }
 
@@ -318,6 +314,7 @@ static int bank_update_impl(const char* fn, const prsink_layout* layout, const B
   int rc = copy_args(fn, layout, bank_kv, cache_kv, n_layers, &g, &do_copy);
   if (rc) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  static_assert(PRSINK_FP_DIM <= 1024, "the blend takes one fingerprint element per thread");
   bank_update_kernel<<<1, 1024, 0, st>>>(bank_phi, bank_src, bank_count, M, phi_b, b, pol,
                                          action_out, mode_out);
   count_launch();
