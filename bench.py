@@ -233,6 +233,55 @@ def attention_alone(name: str, warmup: int, steps: int, repeat: bool = False, nb
     return rec
 
 
+def fused_alone(name: str, warmup: int, steps: int):
+    """prsink_attention_fused (append folded in, sinks read pre-rotated) and the rotation pass
+    prsink_rotate_sinks, each timed alone at a workload's full size on two alternating input
+    sets (each larger than L2)."""
+    import torch
+
+    import pose_retrieved_kv_b200 as P
+    import synth
+
+    cfg = synth.preset(name, block_index=1000, valid_mask=0xFF)
+    lay = P.make_layout(**cfg)
+    _, lblk, _, T = P.prsink_layout_tokens(lay)
+    H, d = cfg["n_heads"], cfg["head_dim"]
+    sets = []
+    for i in range(2):
+        k = synth.normal_bf16((H, T, d), 5 + i, 1).cuda()
+        kr = torch.empty_like(k)
+        P.prsink_rotate_sinks(lay, k, kr, 0xFFFF)
+        sets.append(dict(q=synth.normal_bf16((lblk, H, d), 5 + i, 0).cuda(), k=k,
+                         v=synth.normal_bf16((H, T, d), 5 + i, 2).cuda(), kr=kr,
+                         kn=synth.normal_bf16((lblk, H, d), 5 + i, 3).cuda(),
+                         vn=synth.normal_bf16((lblk, H, d), 5 + i, 4).cuda()))
+    out = torch.empty((lblk, H, d), dtype=torch.bfloat16, device="cuda")
+
+    def fused(i):
+        x = sets[i % 2]
+        P.prsink_attention_fused(lay, x["q"], x["kn"], x["vn"], x["kr"], x["k"], x["v"], out)
+
+    ring = ((1 << cfg["ring_slots"]) - 1) << P.SLOT_RING0
+
+    def rotate(i):
+        x = sets[i % 2]
+        P.prsink_rotate_sinks(lay, x["k"], x["kr"], ring)
+
+    ms_f = time_launches(fused, warmup, steps)
+    ms_r = time_launches(rotate, warmup, steps)
+    if P.prsink_sync_status() != P.PRSINK_OK:
+        raise RuntimeError("device status reported a timeout")
+    peaks = _peaks()
+    rec = _summary(ms_f, 4.0 * lblk * T * d * H, "TFLOP/s", peaks["bf16"],
+                   f"{peaks['source']} bf16_tflops (burst)")
+    n_rot = (cfg["ring_slots"] - 1) * lblk * H             # the two older ring slots
+    rot = _summary(ms_r, 2.0 * n_rot * d * 2, "GB/s", peaks["hbm"], f"{peaks['source']} hbm_gbs")
+    rot["rows_per_call"] = n_rot
+    rec.update(queries=lblk, keys=T, note="includes the raw store of the block into its ring "
+               "slot (the append); sinks read from the rotated copy")
+    return rec, rot
+
+
 def append_alone(name: str, warmup: int, steps: int):
     """prsink_kv_append of one block into a ring slot, timed alone: six source blocks and two
     caches rotate, so consecutive launches touch different memory."""
@@ -305,6 +354,7 @@ def kernel_records(st, args):
            "attention_480x480_repeat": attention_alone("480x480", w, k, repeat=True)}
     for name in ("384x672", "384x672_r4", "672x384"):
         rec[f"attention_{name}"] = attention_alone(name, w, k)
+    rec["attention_fused_480x480"], rec["rotate_ring_slots_480x480"] = fused_alone("480x480", w, k)
     rec["note"] = ("attention: burst bf16 peak (a kernel timed alone); 'rotating' alternates "
                    "two input sets of 322 MB, 'repeat' reuses one (K/V of 295 MB exceed the "
                    "126 MB L2 either way)")
@@ -340,29 +390,82 @@ def _inputs(args, cfg_full, rank, world, dev):
 
 def _block(st, P, b, kp_dev, ok_dev, qkv, out, events=None, stream=None):
     """One block of the stream: retrieval + dynamic fill, per layer 3 denoising passes and the
-    Clean KV Update pass (append + attention), bank update."""
+    Clean KV Update pass (append + attention), bank update.  Fused streams run each pass as one
+    prsink_attention_fused launch (after the layer's once-per-block rotation pass).  ``events``
+    collects the attention launch of every pass (the fused launch includes the append)."""
     import torch
     st.begin_block(kp_dev[b], ok_dev[b])
     i = 0
     pool = len(qkv)
     for layer in range(st.n_layers):
+        st.prepare_layer(layer)
         for p in range(PASSES):
             q, kn, vn = qkv[(b * st.n_layers * PASSES + i) % pool]
             i += 1
             lay = st.layout()
             k, v = st.kv(layer)
-            P.prsink_kv_append(lay, kn, vn, k, v, P.SLOT_RING0 + st.b % st.R)
-            if p == PASSES - 1 and st.b == 0:
-                P.prsink_kv_append(lay, kn, vn, k, v, P.SLOT_STATIC)
+            if not st.fused:
+                P.prsink_kv_append(lay, kn, vn, k, v, P.SLOT_RING0 + st.b % st.R)
             if events is not None:
                 e0 = torch.cuda.Event(enable_timing=True)
                 e1 = torch.cuda.Event(enable_timing=True)
                 e0.record(stream)
-            P.prsink_attention(lay, q, k, v, out, None, st.dyn_src)
+            if st.fused:
+                P.prsink_attention_fused(lay, q, kn, vn, st.k_rot[layer], k, v, out, None,
+                                         st.dyn_src)
+            else:
+                P.prsink_attention(lay, q, k, v, out, None, st.dyn_src)
             if events is not None:
                 e1.record(stream)
                 events.append((e0, e1))
+            if p == PASSES - 1 and st.b == 0:
+                P.prsink_kv_append(lay, kn, vn, k, v, P.SLOT_STATIC)
+                if st.fused:
+                    st.mark_written(layer, P.SLOT_STATIC)
     st.end_block()
+
+
+def step_record(cfg, fused: bool, qkv, ref, kp_dev, ok_dev, dev, steps: int = 5,
+                warmup: int = 3):
+    """The per-block step on a stream of its own with the given path (fused: one
+    prsink_attention_fused launch per pass after a rotation pass per layer and block; unfused:
+    append + prsink_attention), timed in the steady state after the bank was filled."""
+    import torch
+
+    import pose_retrieved_kv_b200 as P
+
+    n_layers = len(ref)
+    st = P.PRSinkStream(cfg, n_layers=n_layers, M=M_BANK, write_blocks=WRITE_BLOCKS, device=dev,
+                        fused=fused)
+    for layer in range(n_layers):
+        st.set_ref(layer, ref[layer], ref[layer])
+    lblk, T, H, d = st.L_blk, st.T, cfg["n_heads"], cfg["head_dim"]
+    out = torch.empty((lblk, H, d), dtype=torch.bfloat16, device=dev)
+    for b in range(WRITE_BLOCKS + warmup):
+        _block(st, P, b, kp_dev, ok_dev, qkv, out)
+    ev = []
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for k in range(steps):
+        _block(st, P, WRITE_BLOCKS + warmup + k, kp_dev, ok_dev, qkv, out, ev)
+    t1.record()
+    torch.cuda.synchronize()
+    if P.prsink_sync_status() != P.PRSINK_OK:
+        raise RuntimeError("device status reported a timeout")
+    ms = t0.elapsed_time(t1) / steps
+    attn = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    tf = 4.0 * lblk * T * d * H / (attn / 1e3) / 1e12
+    peaks = _peaks()
+    del st
+    torch.cuda.empty_cache()
+    return {"path": "fused" if fused else "unfused", "ms_per_step": round(ms, 3),
+            "layer_blocks_per_s": round(n_layers * 1e3 / ms, 3),
+            "attention_avg_ms": round(attn, 4), "attention_tflops": round(tf, 1),
+            "frac_of_bf16_sustained": round(tf / peaks["bf16_sustained"], 4),
+            "note": "fused: the timed launch includes the append; the rotation pass (once per "
+                    "layer and block) is in ms_per_step only"}
 
 
 def run_stream(st, P, kp_dev, ok_dev, qkv, out, n_blocks, dev):
@@ -412,7 +515,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     cfg = shard.shard_config(cfg_full, world, rank) if split else cfg_full
     n_layers = args.layers
     H, d = cfg["n_heads"], cfg["head_dim"]
-    st = P.PRSinkStream(cfg, n_layers=n_layers, M=M_BANK, write_blocks=WRITE_BLOCKS, device=dev)
+    st = P.PRSinkStream(cfg, n_layers=n_layers, M=M_BANK, write_blocks=WRITE_BLOCKS, device=dev,
+                        fused=args.path == "fused")
     lblk, T = st.L_blk, st.T
     qkv, ref, pose_seed = _inputs(args, cfg_full, rank, world, dev)
     for layer in range(n_layers):
@@ -479,6 +583,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     extras = stream_rec = None
     if world == 1 and not args.no_extras:
         extras = kernel_records(st, args)
+        extras["step_other_path"] = step_record(cfg, args.path != "fused", qkv, ref, kp_dev,
+                                                ok_dev, dev)
         stream_rec = run_stream(st, P, kp_dev, ok_dev, qkv, out, args.stream_blocks, dev)
 
     if rank != 0:
@@ -498,6 +604,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "config": {"workload": f"per-block step {args.config}: {n_layers} layers x "
                                f"({PASSES - 1} denoise + 1 clean) x (append + PR-Sink attention), "
                                "retrieval + dynamic fill, bank update",
+                   "path": args.path,
                    "heads": cfg_full["n_heads"], "heads_per_gpu": H, "head_dim": d,
                    "queries": lblk, "keys": T, "ring_slots": cfg["ring_slots"],
                    "layers": n_layers, "bank": M_BANK,
@@ -761,6 +868,9 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default="480x480",
                     choices=["480x480", "384x672", "384x672_r4", "672x384", "stream300"])
+    ap.add_argument("--path", choices=["fused", "unfused"], default="unfused",
+                    help="fused: each pass is one prsink_attention_fused launch (append folded "
+                         "in, sinks pre-rotated once per layer and block)")
     ap.add_argument("--partition", choices=["heads", "replicas"], default="heads",
                     help="N > 1: split the heads of one stream, or one stream per GPU")
     ap.add_argument("--layers", type=int, default=40)

@@ -106,6 +106,47 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// Softmax exponentials on the FMA pipe for a share of the score columns, so that the
+// special-function unit (16 results per clock per SM, exactly the rate the tensor core produces
+// scores) is not the limit.  Column pair i (0..15) of every 32-column chunk uses the polynomial
+// when bit i of kPolyPairs is set.
+#ifndef PRSINK_POLY_PAIRS
+#define PRSINK_POLY_PAIRS 0x8888
+#endif
+constexpr uint32_t kPolyPairs = PRSINK_POLY_PAIRS;
+#ifndef PRSINK_MAX3
+#define PRSINK_MAX3 1
+#endif
+constexpr bool kMax3 = PRSINK_MAX3;
+
+// 2^x for a pair, by Cody-Waite range reduction (x = n + f, n the nearest integer, taken with the
+// 1.5 * 2^23 rounding constant, f in [-1/2, 1/2]) and a degree-3 polynomial minimising the
+// relative error of 2^f on [-1/2, 1/2] (Remez exchange; pose_retrieved_kv_b200/exp2_poly.py
+// derives the coefficients; relative error below 1.5e-4 in float32, far under the bf16
+// rounding of P that follows).  2^n is added to the exponent field of p(f); x is clamped below
+// at -125 so that field stays positive (2^-125 instead of ~0 is negligible next to the row sum).
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  constexpr float kMagic = 12582912.0f;                // 1.5 * 2^23
+  x.x = fmaxf(x.x, -125.0f);
+  x.y = fmaxf(x.y, -125.0f);
+  const float2 t = fadd2(x, make_float2(kMagic, kMagic));
+  const float2 r = fadd2(t, make_float2(-kMagic, -kMagic));      // round(x), exact
+  const float2 f = ffma2(r, make_float2(-1.0f, -1.0f), x);       // x - round(x), exact
+  float2 q = ffma2(make_float2(0.0551716685295105f, 0.0551716685295105f), f,
+                   make_float2(0.2426111251115799f, 0.2426111251115799f));
+  q = ffma2(q, f, make_float2(0.6932609677314758f, 0.6932609677314758f));
+  q = ffma2(q, f, make_float2(0.9999280571937561f, 0.9999280571937561f));
+  // exponent: the low bits of t hold n; (bits(t) << 23) mod 2^32 = n << 23
+  return make_float2(__uint_as_float(__float_as_uint(q.x) + __float_as_uint(t.x) * 8388608u),
+                     __uint_as_float(__float_as_uint(q.y) + __float_as_uint(t.y) * 8388608u));
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float y;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(y) : "f"(a), "f"(b), "f"(c));
+  return y;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&b);
@@ -731,10 +772,20 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
       float mx[8];
 #pragma unroll
       for (int a = 0; a < 8; ++a) mx[a] = __uint_as_float(s[a]);
+      if constexpr (kMax3) {
 #pragma unroll
-      for (int c = 8; c < 128; c += 8)
+        for (int c = 8; c < 120; c += 16)
 #pragma unroll
-        for (int a = 0; a < 8; ++a) mx[a] = fmaxf(mx[a], __uint_as_float(s[c + a]));
+          for (int a = 0; a < 8; ++a)
+            mx[a] = fmax3(mx[a], __uint_as_float(s[c + a]), __uint_as_float(s[c + 8 + a]));
+#pragma unroll
+        for (int a = 0; a < 8; ++a) mx[a] = fmaxf(mx[a], __uint_as_float(s[120 + a]));
+      } else {
+#pragma unroll
+        for (int c = 8; c < 128; c += 8)
+#pragma unroll
+          for (int a = 0; a < 8; ++a) mx[a] = fmaxf(mx[a], __uint_as_float(s[c + a]));
+      }
       const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
                              fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * p.scale_log2;
       float alpha = 1.f;
@@ -759,7 +810,8 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
           const int c = ch * 32 + 2 * i;
           const float2 e2 = ffma2(make_float2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])),
                                   scale2, negm);
-          const float2 pr = make_float2(ex2(e2.x), ex2(e2.y));
+          const float2 pr = ((kPolyPairs >> i) & 1u) ? exp2_poly2(e2)
+                                                      : make_float2(ex2(e2.x), ex2(e2.y));
           sum2[i & 3] = fadd2(sum2[i & 3], pr);
           pk[i] = pack_bf16(pr.x, pr.y);
         }

@@ -104,7 +104,7 @@ class PRSinkStream:
     def set_ref(self, layer: int, k_ref, v_ref, stream=None):
         k, v = self.kv(layer)
         L.prsink_kv_append(self.layout(), k_ref, v_ref, k, v, L.SLOT_REF, stream)
-        self._rot_pending[layer] |= 1 << L.SLOT_REF
+        self.mark_written(layer, L.SLOT_REF)
 
     def begin_block(self, kp, frame_ok, stream=None):
         """Fingerprint (kp f32 [3][62][3], frame_ok u8 [3], on the device) and retrieval."""
@@ -120,6 +120,25 @@ class PRSinkStream:
                           self.bank_count, self.M, self.b - 1, self.r, self.score, self.copied,
                           self.dyn_src, self.bank_kv, self.cache_kv, self.n_layers, stream)
 
+    def mark_written(self, layer: int, slot: int):
+        """Fused mode: a fixed-position slot (ref, static) of ``layer`` was written outside
+        ``layer_pass``; its rotated copy is refreshed by the next ``prepare_layer``."""
+        self._rot_pending[layer] |= 1 << int(slot)
+
+    def prepare_layer(self, layer: int, stream=None):
+        """Fused mode: refresh the layer's rotated sink keys once per block (ring slots move one
+        rank per block; the dynamic slot when retrieval refilled it; ref and static once after
+        they were written).  Called by ``layer_pass``; a no-op when unfused or already done."""
+        if not self.fused or self._rot_block[layer] == self.b:
+            return
+        k, _ = self.kv(layer)
+        ring = ((1 << self.R) - 1) << L.SLOT_RING0
+        mask = ring | (1 << L.SLOT_DYNAMIC) | self._rot_pending[layer]
+        L.prsink_rotate_sinks(self.layout(), k, self.k_rot[layer], mask, self.copied,
+                              self.dyn_src, stream)
+        self._rot_pending[layer] = 0
+        self._rot_block[layer] = self.b
+
     def layer_pass(self, layer: int, q, k_new, v_new, out, lse=None, clean: bool = False,
                    stream=None):
         """Append this pass's raw K/V into ring slot b mod R (and, on block 0's clean pass,
@@ -127,20 +146,12 @@ class PRSinkStream:
         lay = self.layout()
         k, v = self.kv(layer)
         if self.fused:
-            if self._rot_block[layer] != self.b:
-                # ring slots move one rank per block; the dynamic slot when retrieval refilled
-                # it; ref and static once after they were written
-                ring = ((1 << self.R) - 1) << L.SLOT_RING0
-                mask = ring | (1 << L.SLOT_DYNAMIC) | self._rot_pending[layer]
-                L.prsink_rotate_sinks(lay, k, self.k_rot[layer], mask, self.copied,
-                                      self.dyn_src, stream)
-                self._rot_pending[layer] = 0
-                self._rot_block[layer] = self.b
+            self.prepare_layer(layer, stream)
             L.prsink_attention_fused(lay, q, k_new, v_new, self.k_rot[layer], k, v, out, lse,
                                      self.dyn_src, stream)
             if clean and self.b == 0:
                 L.prsink_kv_append(lay, k_new, v_new, k, v, L.SLOT_STATIC, stream)
-                self._rot_pending[layer] |= 1 << L.SLOT_STATIC
+                self.mark_written(layer, L.SLOT_STATIC)
             return
         L.prsink_kv_append(lay, k_new, v_new, k, v, L.SLOT_RING0 + self.b % self.R, stream)
         if clean and self.b == 0:
