@@ -112,6 +112,30 @@ int prsink_attention(const prsink_layout* layout, const void* q, const void* k_c
                      const void* v_cache, void* out, float* lse, const long long* dyn_src,
                      void* stream);
 
+/* prsink_attention with the last wave split over the key range (same result, up to float
+ * rounding of the split sums).
+ *
+ * One CTA per SM computes a unit = (head, 256 queries).  When the units leave the last wave of
+ * the device (#SM units per wave) nearly empty (384x672: 480 units = 3 waves of 148 + 36), each
+ * of the r units of that wave runs as S = min(#SM / r, 8) CTAs over equal shares of the key
+ * tiles; each writes its unnormalised partial (float32 O, running max, sum) to `scratch`, and
+ * the last one to finish combines them (O = sum_s O_s 2^(m_s - M) / sum_s l_s 2^(m_s - M)).
+ * Arguments as prsink_attention, plus:
+ *   scratch        device memory of at least prsink_attention_scratch_bytes(layout) bytes,
+ *                  256-byte aligned, owned by the caller, not shared with a concurrent call;
+ *                  may be NULL when that size is 0 (no split planned: a plain attention)
+ *   scratch_bytes  its size
+ * The plan depends on the current device's SM count.  The arrival counters inside `scratch` are
+ * cleared on `stream` by each call.  Errors: as prsink_attention; PRSINK_ERR_ARG for a missing,
+ * misaligned or too small scratch. */
+int prsink_attention_split(const prsink_layout* layout, const void* q, const void* k_cache,
+                           const void* v_cache, void* out, float* lse, const long long* dyn_src,
+                           void* scratch, long long scratch_bytes, void* stream);
+
+/* Scratch bytes prsink_attention_split needs for `layout` on the current device (0 when the
+ * last wave is full enough that no split is planned; -1 for an invalid layout). */
+long long prsink_attention_scratch_bytes(const prsink_layout* layout);
+
 /* Rotated copy of the sink keys, for prsink_attention_fused.
  *
  * [digest] weaknesses, point 2: reuse cached work to cut the repeated computation of the Ref and

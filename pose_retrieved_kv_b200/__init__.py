@@ -13,5 +13,6 @@ from ._lib import (  # noqa: F401
     prsink_retrieve, prsink_sync_status, prsink_version, BANK_DECAY, BANK_FROZEN, BANK_GATED,
     BANK_MODE_BLEND, BANK_MODE_NONE, BANK_MODE_STORE, BankPolicy, make_policy,
     prsink_bank_update_policy, prsink_retrieve_fallback, prsink_attention_fused,
-    prsink_rotate_sinks, prsink_debug_attention_stall)
+    prsink_rotate_sinks, prsink_debug_attention_stall, prsink_attention_split,
+    prsink_attention_scratch_bytes)
 from .stream import PRSinkStream, stream_valid_mask  # noqa: F401

@@ -103,6 +103,8 @@ def _load():
         "prsink_retrieve": ([lp, vp, vp, vp, vp, i, ll, vp, vp, vp, vp, vp, vp, i, vp], i),
         "prsink_bank_update": ([lp, vp, vp, vp, i, vp, ll, i, vp, vp, vp, i, vp], i),
         "prsink_attention_fused": ([lp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp], i),
+        "prsink_attention_split": ([lp, vp, vp, vp, vp, vp, vp, vp, ll, vp], i),
+        "prsink_attention_scratch_bytes": ([lp], ll),
         "prsink_rotate_sinks": ([lp, vp, vp, ctypes.c_uint, vp, vp, vp], i),
         "prsink_retrieve_fallback": ([lp, vp, vp, i, vp, vp, vp, i, ll, vp, vp, vp, vp, vp, vp,
                                       i, vp], i),
@@ -127,7 +129,8 @@ def exported_symbols() -> list:
             "prsink_attention", "prsink_kv_append", "prsink_fingerprint", "prsink_retrieve",
             "prsink_bank_update", "prsink_sync_status", "prsink_debug_wait_timeout",
             "prsink_retrieve_fallback", "prsink_bank_update_policy", "prsink_attention_fused",
-            "prsink_rotate_sinks", "prsink_debug_attention_stall"]
+            "prsink_rotate_sinks", "prsink_debug_attention_stall", "prsink_attention_split",
+            "prsink_attention_scratch_bytes"]
 
 
 def _check(rc: int, fn: str):
@@ -209,6 +212,30 @@ def prsink_attention(layout: Layout, q, k_cache, v_cache, out, lse=None, dyn_src
         _ptr(lse, "lse", torch.float32, H * lblk), _ptr(dyn_src, "dyn_src", torch.int64, 1),
         _stream(stream))
     _check(rc, "prsink_attention")
+
+
+def prsink_attention_scratch_bytes(layout: Layout) -> int:
+    n = _lib.prsink_attention_scratch_bytes(ctypes.byref(layout))
+    if n < 0:
+        raise PRSinkError(PRSINK_ERR_ARG, "prsink_attention_scratch_bytes", prsink_last_error())
+    return n
+
+
+def prsink_attention_split(layout: Layout, q, k_cache, v_cache, out, scratch, lse=None,
+                           dyn_src=None, stream=None):
+    """``scratch``: a uint8 CUDA tensor of at least prsink_attention_scratch_bytes bytes (None
+    when that is 0)."""
+    _, lblk, _, T = prsink_layout_tokens(layout)
+    H, d = layout.n_heads, layout.head_dim
+    rc = _lib.prsink_attention_split(
+        ctypes.byref(layout), _ptr(q, "q", torch.bfloat16, lblk * H * d),
+        _ptr(k_cache, "k_cache", torch.bfloat16, H * T * d),
+        _ptr(v_cache, "v_cache", torch.bfloat16, H * T * d),
+        _ptr(out, "out", torch.bfloat16, lblk * H * d),
+        _ptr(lse, "lse", torch.float32, H * lblk), _ptr(dyn_src, "dyn_src", torch.int64, 1),
+        _ptr(scratch, "scratch", torch.uint8),
+        0 if scratch is None else int(scratch.numel()), _stream(stream))
+    _check(rc, "prsink_attention_split")
 
 
 def prsink_attention_fused(layout: Layout, q, k_new, v_new, k_rot, k_cache, v_cache, out,

@@ -42,6 +42,7 @@ constexpr uint32_t kTmemCols = 512;
 constexpr int kTableMaxBytes = 28 * 1024;
 constexpr int kMaxTiles = 1024;             // key tiles per call (T <= 131072)
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale O when the max grows > 2^8
+constexpr int kMaxSplit = 8;                // split CTAs per unit (key-range shares)
 
 struct Params {
   int H, L_blk, T, L_f, grid_h, grid_w;
@@ -69,6 +70,13 @@ struct Params {
   unsigned rot_mask;
   const int* rot_dyn_flag;              // dynamic slot rotated only if *flag != 0 (nullable)
   int debug_stall;                      // self-test: withhold the first S commit of query tile 0
+  // work decomposition (1-D grid): units = (head, pair of query tiles), nqb per head, head-major;
+  // units >= split_base run as n_split CTAs, each over an equal share of the live key tiles,
+  // writing unnormalised partial results that the last of them combines
+  int nqb, split_base, n_split;
+  float* part_o;                        // [split units][n_split][NQ * BM][D] float32
+  float2* part_ml;                      // [split units][n_split][NQ * BM] (max in log2 units, sum)
+  int* part_cnt;                        // [split units] arrival counters (zero at launch)
 };
 
 // Entries of the per-CTA tile list: a key tile index and what the roles do with it.
@@ -415,6 +423,8 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
   __shared__ uint16_t tile_list[kMaxTiles];      // live tiles in order (kTile* bits)
   __shared__ int n_live_s;
   __shared__ int last_k_s, last_v_s;             // last K / V loads issued (for the drain)
+  __shared__ int list_off_s;                     // first tile of this CTA's share
+  __shared__ int combine_s;                      // this CTA combines the split partials
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t raw = smem_u32(dsmem);
@@ -424,8 +434,15 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
   float2* tab = reinterpret_cast<float2*>(gb + LY::kTab);
   auto bar = [&](int i) { return smem_u32(&bars[i]); };
 
-  const int q0 = blockIdx.x * (NQ * BM);
-  const int h = blockIdx.y;
+  int unit = blockIdx.x, split = 0, n_split = 1;
+  if (unit >= p.split_base) {
+    const int k = unit - p.split_base;
+    n_split = p.n_split;
+    unit = p.split_base + k / n_split;
+    split = k % n_split;
+  }
+  const int h = unit / p.nqb, qb = unit % p.nqb;
+  const int q0 = qb * (NQ * BM);
 
   if (threadIdx.x == 0) {
     mbar_init(bar(B_QFULL), 1);
@@ -492,13 +509,19 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
       for (int i = lane; i < p.n_cur_tiles; i += 32) {
         uint16_t e = static_cast<uint16_t>(i) | kTileNew;
         if ((i + 1) * BN > p.L_blk) e |= kTileMask;
-        if (i % static_cast<int>(gridDim.x) == static_cast<int>(blockIdx.x))
+        if (i % p.nqb == qb)
           e |= kTileStore | kTileVfix;
         tile_list[base + i] = e;
       }
       base += p.n_cur_tiles;
     }
-    if (lane == 0) n_live_s = base;
+    if (lane == 0) {
+      // a split CTA takes an equal share of the live tiles
+      const int j0 = static_cast<int>(static_cast<long long>(base) * split / n_split);
+      const int j1 = static_cast<int>(static_cast<long long>(base) * (split + 1) / n_split);
+      list_off_s = j0;
+      n_live_s = j1 - j0;
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -508,6 +531,7 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
   const unsigned vm = vmask_s;
   const uint64_t deadline = globaltimer() + p.timeout_ns;
   const int n_live = n_live_s;
+  const uint16_t* tiles = tile_list + list_off_s;
 
   if (warp >= kProducerWarp) {
     setmaxnreg_dec<80>();
@@ -520,7 +544,7 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
                       q0 + qt * BM);
       int j = 0, last_k = -1, last_v = -1;               // last iterations whose loads went out
       for (; j < n_live; ++j) {
-        const uint16_t te = tile_list[j];
+        const uint16_t te = tiles[j];
         const int n = te & kTileIdx;
         const bool cur = kFused && (te & kTileNew);    // [tokens][H][d] map: (d, head, token)
         const int c1 = cur ? h : n * BN, c2 = cur ? n * BN : h;
@@ -575,7 +599,7 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
       int j = 0;
       bool prev_partial = false;
       for (; ok && j < n_live; ++j) {
-        const bool partial = tile_list[j] & kTileVfix;    // V touched by the rotation warps
+        const bool partial = tiles[j] & kTileVfix;        // V touched by the rotation warps
         const int st = j & 1;
         // P0(j-1).V(j-1) does not need K(j): issue it before waiting for the rotation
         if (j >= 1 && !pv_mma(0, j - 1, prev_partial)) { ok = false; break; }
@@ -628,7 +652,7 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
       int cur = -2 * BN, s_cur = 0, frame = 0, y = 0, x = 0;   // no previous row yet
       int n_stored = 0;                                         // raw K tiles stored so far
       for (int j = 0; j < n_live; ++j) {
-        const uint16_t te = tile_list[j];
+        const uint16_t te = tiles[j];
         const int n = te & kTileIdx;
         const int st = j & 1;
         const uint32_t kt = sK + st * LY::kTileBytes;
@@ -724,7 +748,7 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
     int j = 0;
     bool ok = true;
     for (; j < n_live; ++j) {
-      const uint16_t te = tile_list[j];
+      const uint16_t te = tiles[j];
       const int n = te & kTileIdx;
       ok = mbar_wait(bar(B_SFULL + qt), j & 1, &ab, deadline, p.status);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }   // tcgen05.ld is warp-collective
@@ -847,6 +871,12 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
       inv = l > 0.f ? 1.f / l : 0.f;
     }
     __nv_bfloat16* orow = p.out + (static_cast<size_t>(qi) * p.H + h) * D;
+    // a split CTA writes its unnormalised partial (O, max, sum) for the combine instead
+    const size_t slot = static_cast<size_t>(unit - p.split_base) * n_split + split;
+    float* prow = n_split > 1 ? p.part_o + (slot * (NQ * BM) + qt * BM + t) * D : nullptr;
+    if (n_split > 1)
+      p.part_ml[slot * (NQ * BM) + qt * BM + t] =
+          have ? make_float2(m, l) : make_float2(-INFINITY, 0.f);
 #pragma unroll 1
     for (int cc = 0; cc < D / 32; ++cc) {
       uint32_t o[32];
@@ -857,7 +887,12 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
         for (int i = 0; i < 32; ++i) o[i] = 0u;
       }
-      if (qi < p.L_blk) {
+      if (prow) {
+#pragma unroll
+        for (int i = 0; i < 32; i += 4)
+          *reinterpret_cast<uint4*>(prow + cc * 32 + i) = make_uint4(o[i], o[i + 1], o[i + 2],
+                                                                     o[i + 3]);
+      } else if (qi < p.L_blk) {
 #pragma unroll
         for (int i = 0; i < 32; i += 8) {
           uint4 v;
@@ -869,9 +904,10 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
         }
       }
     }
-    if (p.lse && qi < p.L_blk)
+    if (p.lse && qi < p.L_blk && n_split == 1)
       p.lse[static_cast<size_t>(h) * p.L_blk + qi] =
           have ? (m + log2f(l)) * 0.69314718055994530942f : -INFINITY;
+    if (n_split > 1) __threadfence();   // partials visible before this CTA's arrival counts
   }
 
   tc_fence_before();
@@ -897,6 +933,58 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
   if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
+  }
+  if (n_split > 1) {
+    // the last of a unit's split CTAs to arrive combines their partials:
+    //   M = max_s m_s,  L = sum_s l_s 2^(m_s - M),  O = sum_s O_s 2^(m_s - M) / L
+    const size_t k = static_cast<size_t>(unit - p.split_base);
+    if (threadIdx.x == 0) {
+      __threadfence();
+      combine_s = atomicAdd(&p.part_cnt[k], 1) == n_split - 1;
+    }
+    __syncthreads();
+    if (combine_s) {
+      __threadfence();
+      const int r = threadIdx.x;                  // one row per thread
+      const int qi = q0 + r;
+      if (r < NQ * BM && qi < p.L_blk) {
+        const float2* ml = p.part_ml + k * n_split * (NQ * BM) + r;
+        float M = -INFINITY;
+        for (int sp = 0; sp < n_split; ++sp) M = fmaxf(M, __ldcg(ml + sp * (NQ * BM)).x);
+        // weight of share sp: 2^(m_s - M), 0 for a share without keys (or no keys at all)
+        auto weight = [&](int sp) {
+          const float ms = __ldcg(ml + sp * (NQ * BM)).x;
+          return ms > -INFINITY ? ex2(ms - M) : 0.f;
+        };
+        float L = 0.f;
+        for (int sp = 0; sp < n_split; ++sp) L += weight(sp) * __ldcg(ml + sp * (NQ * BM)).y;
+        const float inv = L > 0.f ? 1.f / L : 0.f;
+        __nv_bfloat16* orow = p.out + (static_cast<size_t>(qi) * p.H + h) * D;
+        const float* o0 = p.part_o + (k * n_split * (NQ * BM) + r) * D;
+#pragma unroll 1
+        for (int c = 0; c < D; c += 8) {
+          float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+          for (int sp = 0; sp < n_split; ++sp) {
+            const float w = weight(sp);
+            const float4* src =
+                reinterpret_cast<const float4*>(o0 + static_cast<size_t>(sp) * (NQ * BM) * D + c);
+            const float4 a = __ldcg(src), b = __ldcg(src + 1);
+            acc[0] += w * a.x; acc[1] += w * a.y; acc[2] += w * a.z; acc[3] += w * a.w;
+            acc[4] += w * b.x; acc[5] += w * b.y; acc[6] += w * b.z; acc[7] += w * b.w;
+          }
+          uint4 v;
+          v.x = pack_bf16(acc[0] * inv, acc[1] * inv);
+          v.y = pack_bf16(acc[2] * inv, acc[3] * inv);
+          v.z = pack_bf16(acc[4] * inv, acc[5] * inv);
+          v.w = pack_bf16(acc[6] * inv, acc[7] * inv);
+          *reinterpret_cast<uint4*>(orow + c) = v;
+        }
+        if (p.lse)
+          p.lse[static_cast<size_t>(h) * p.L_blk + qi] =
+              L > 0.f ? (M + log2f(L)) * 0.69314718055994530942f : -INFINITY;
+      }
+      if (threadIdx.x == 0) p.part_cnt[k] = 0;   // ready for the next launch
+    }
   }
 }
 
@@ -1131,8 +1219,9 @@ static int launch(const prsink_layout* L, const Geometry& g, const Buffers& b, P
   static int allowed[64] = {0};
   rc = allow_smem(prsink_attention_kernel<D, RT, RH, kFused>, smem, allowed, what);
   if (rc) return rc;
-  dim3 grid((g.L_blk + NQ * BM - 1) / (NQ * BM), L->n_heads);
-  prsink_attention_kernel<D, RT, RH, kFused><<<grid, kThreads, smem, st>>>(mq, mk, mv, mkn, mvn,
+  const int units = p.nqb * L->n_heads;
+  const int ctas = p.split_base + (units - p.split_base) * p.n_split;
+  prsink_attention_kernel<D, RT, RH, kFused><<<ctas, kThreads, smem, st>>>(mq, mk, mv, mkn, mvn,
                                                                           mks, mvs, p);
   count_launch();
   return check_launch(what);
@@ -1165,6 +1254,44 @@ static int launch_rotate(const prsink_layout* L, const Geometry& g, const void* 
   prsink_rotate_kernel<D, RT, RH><<<grid, kRotThreads, smem, st>>>(ms, md, p);
   count_launch();
   return check_launch("prsink_rotate_sinks");
+}
+
+// Split of the last wave.  Units (head, pair of query tiles) run one CTA per SM; when the
+// last wave holds r < #SM units, each of those runs as S = min(#SM / r, kMaxSplit) CTAs over
+// equal shares of the key tiles, so the last wave takes ~1/S of a unit's time.
+struct SplitPlan {
+  int split_base, n_split, r;
+  size_t o_bytes, ml_bytes, cnt_bytes;       // scratch regions, each 256-byte aligned
+  size_t total() const { return o_bytes + ml_bytes + cnt_bytes; }
+};
+
+static size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+static SplitPlan plan_split(const Geometry& g, int H, int D) {
+  SplitPlan sp{};
+  const int nqb = static_cast<int>((g.L_blk + NQ * BM - 1) / (NQ * BM));
+  const int units = nqb * H;
+  int n_sm = 148, dev = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
+  sp.split_base = units;
+  sp.n_split = 1;
+  if (units <= 0 || n_sm <= 0) return sp;
+  const int waves = (units + n_sm - 1) / n_sm;
+  const int r = units - (waves - 1) * n_sm;
+  int S = n_sm / r;
+  if (S > kMaxSplit) S = kMaxSplit;
+  const int tiles = static_cast<int>((g.T + BN - 1) / BN);
+  if (S > tiles) S = tiles;
+  if (S < 2) return sp;
+  sp.split_base = units - r;
+  sp.n_split = S;
+  sp.r = r;
+  const size_t parts = static_cast<size_t>(r) * S * (NQ * BM);
+  sp.o_bytes = align256(parts * D * sizeof(float));
+  sp.ml_bytes = align256(parts * sizeof(float2));
+  sp.cnt_bytes = align256(static_cast<size_t>(r) * sizeof(int));
+  return sp;
 }
 
 // Self-test of the attention kernel's abort path (per host thread, one call).
@@ -1230,6 +1357,9 @@ static int fill_params(const prsink_layout* layout, const Geometry& g, Params& p
   p.status = status_word_ptr();
   p.timeout_ns = 2000000000ull;
   p.cur_slot = -1;
+  p.nqb = static_cast<int>((g.L_blk + NQ * BM - 1) / (NQ * BM));
+  p.split_base = p.nqb * layout->n_heads;     // no split unless a caller plans one
+  p.n_split = 1;
   if (g_debug_stall_ns > 0) {           // armed by prsink_debug_attention_stall: one call only
     p.debug_stall = 1;
     p.timeout_ns = static_cast<unsigned long long>(g_debug_stall_ns);
@@ -1299,6 +1429,60 @@ extern "C" int prsink_attention(const prsink_layout* layout, const void* q, cons
   if (g.L_blk == 0) return PRSINK_OK;
   const Buffers b{q, k_cache, v_cache, nullptr, nullptr, nullptr, nullptr};
   return dispatch<false>(layout, g, b, p, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" long long prsink_attention_scratch_bytes(const prsink_layout* layout) {
+  using namespace prsink::attn;
+  Geometry g;
+  if (geometry(layout, &g)) return -1;
+  return static_cast<long long>(plan_split(g, layout->n_heads, layout->head_dim).total());
+}
+
+// Shared by the split entry points: plan, carve `scratch` and launch.
+static int attention_split_impl(const char* what, const prsink_layout* layout, const void* q,
+                                const void* k_cache, const void* v_cache, void* out, float* lse,
+                                const long long* dyn_src, void* scratch,
+                                long long scratch_bytes, void* stream) {
+  using namespace prsink::attn;
+  Geometry g;
+  int rc = check_attention_args(layout, &g, what, {q, k_cache, v_cache, out}, lse);
+  if (rc) return rc;
+  Params p;
+  rc = fill_params(layout, g, p, what);
+  if (rc) return rc;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.dyn_src = dyn_src;
+  if (g.L_blk == 0) return PRSINK_OK;
+  const SplitPlan sp = plan_split(g, layout->n_heads, layout->head_dim);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (sp.n_split > 1) {
+    if (!scratch || (reinterpret_cast<uintptr_t>(scratch) & 255u) ||
+        scratch_bytes < static_cast<long long>(sp.total())) {
+      set_error("%s: scratch must be 256-byte aligned and hold %zu bytes (got %lld)", what,
+                sp.total(), scratch_bytes);
+      return PRSINK_ERR_ARG;
+    }
+    char* base = static_cast<char*>(scratch);
+    p.part_o = reinterpret_cast<float*>(base);
+    p.part_ml = reinterpret_cast<float2*>(base + sp.o_bytes);
+    p.part_cnt = reinterpret_cast<int*>(base + sp.o_bytes + sp.ml_bytes);
+    p.split_base = sp.split_base;
+    p.n_split = sp.n_split;
+    // the arrival counters start at zero (the combining CTA also resets them)
+    if (cudaMemsetAsync(p.part_cnt, 0, sp.cnt_bytes, st) != cudaSuccess)
+      return check_launch(what);
+  }
+  const Buffers b{q, k_cache, v_cache, nullptr, nullptr, nullptr, nullptr};
+  return dispatch<false>(layout, g, b, p, st);
+}
+
+extern "C" int prsink_attention_split(const prsink_layout* layout, const void* q,
+                                      const void* k_cache, const void* v_cache, void* out,
+                                      float* lse, const long long* dyn_src, void* scratch,
+                                      long long scratch_bytes, void* stream) {
+  return attention_split_impl("prsink_attention_split", layout, q, k_cache, v_cache, out, lse,
+                              dyn_src, scratch, scratch_bytes, stream);
 }
 
 extern "C" int prsink_attention_fused(const prsink_layout* layout, const void* q,

@@ -141,3 +141,16 @@ def test_copy_buffers_sized_for_the_layout_or_rejected_before_launch():
         P.prsink_retrieve(lay, f32(558), f32(M * 558), i64(M), i32(1), M, 0, i32(1), None,
                           i32(1), i64(1), bf(good_bank), bf(good_cache), n_layers)
     assert P.prsink_launch_count() == before
+
+
+def test_split_scratch_plan_sizes():
+    """The split of the last wave, as planned for a 148-SM device (the count a B200 reports;
+    without a GPU the planner assumes it): 384x672 leaves 36 units in its last wave -> 4 shares
+    each; 480x480 fills its last wave (144 of 148) -> no split."""
+    def size(name, **kw):
+        return P.prsink_attention_scratch_bytes(P.make_layout(**synth.preset(name, **kw)))
+    r, S, rows, d = 36, 4, 256, 128
+    want = r * S * rows * d * 4 + r * S * rows * 8 + 256
+    assert size("384x672") == want
+    assert size("480x480") == 0
+    assert size("480x480", n_heads=5) > 0             # 55 units < 148: every unit split
