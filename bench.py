@@ -203,10 +203,12 @@ def _summary(ms, work, unit, peak, peak_source):
             "frac": round(ach / peak, 4), "peak_source": peak_source}
 
 
-def attention_alone(name: str, warmup: int, steps: int, repeat: bool = False, nbuf: int = 2):
+def attention_alone(name: str, warmup: int, steps: int, repeat: bool = False, nbuf: int = 2,
+                    split: bool = False):
     """One attention call at a workload's full size (block 1000, every slot valid), timed
     alone.  ``repeat`` = the same inputs every launch; otherwise ``nbuf`` input sets (each
-    larger than L2) alternate."""
+    larger than L2) alternate.  ``split``: prsink_attention_split (the last wave's units split
+    over the key range)."""
     import torch
 
     import pose_retrieved_kv_b200 as P
@@ -221,14 +223,22 @@ def attention_alone(name: str, warmup: int, steps: int, repeat: bool = False, nb
     k = [synth.normal_bf16((H, T, d), 5 + i, 1).cuda() for i in range(n)]
     v = [synth.normal_bf16((H, T, d), 5 + i, 2).cuda() for i in range(n)]
     out = torch.empty((lblk, H, d), dtype=torch.bfloat16, device="cuda")
-    ms = time_launches(lambda i: P.prsink_attention(lay, q[i % n], k[i % n], v[i % n], out),
-                       warmup, steps)
+    nbytes = P.prsink_attention_scratch_bytes(lay) if split else 0
+    scratch = torch.empty(nbytes, dtype=torch.uint8, device="cuda") if nbytes else None
+    if split:
+        def launch(i):
+            P.prsink_attention_split(lay, q[i % n], k[i % n], v[i % n], out, scratch)
+    else:
+        def launch(i):
+            P.prsink_attention(lay, q[i % n], k[i % n], v[i % n], out)
+    ms = time_launches(launch, warmup, steps)
     if P.prsink_sync_status() != P.PRSINK_OK:
         raise RuntimeError("device status reported a timeout")
     peaks = _peaks()
     rec = _summary(ms, 4.0 * lblk * T * d * H, "TFLOP/s", peaks["bf16"],
                    f"{peaks['source']} bf16_tflops (burst)")
     rec.update(queries=lblk, keys=T, gflop=round(4.0 * lblk * T * d * H / 1e9, 1),
+               scratch_bytes=nbytes,
                inputs="repeated" if repeat else f"{n} sets of {(lblk + 2 * T) * H * d * 2 / 1e6:.0f} MB alternating")
     return rec
 
@@ -354,6 +364,7 @@ def kernel_records(st, args):
            "attention_480x480_repeat": attention_alone("480x480", w, k, repeat=True)}
     for name in ("384x672", "384x672_r4", "672x384"):
         rec[f"attention_{name}"] = attention_alone(name, w, k)
+        rec[f"attention_{name}_split"] = attention_alone(name, w, k, split=True)
     rec["attention_fused_480x480"], rec["rotate_ring_slots_480x480"] = fused_alone("480x480", w, k)
     rec["note"] = ("attention: burst bf16 peak (a kernel timed alone); 'rotating' alternates "
                    "two input sets of 322 MB, 'repeat' reuses one (K/V of 295 MB exceed the "
