@@ -505,7 +505,8 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
       base += __popc(live);
     }
     if (kFused) {
-      // the current block's tiles after the sink tiles; tile i is stored by CTA i mod gridDim.x
+      // the current block's tiles after the sink tiles; tile i is stored by the CTA of query
+      // pair i mod nqb
       for (int i = lane; i < p.n_cur_tiles; i += 32) {
         uint16_t e = static_cast<uint16_t>(i) | kTileNew;
         if ((i + 1) * BN > p.L_blk) e |= kTileMask;
