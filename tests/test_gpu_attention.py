@@ -72,9 +72,9 @@ def test_small_3d_every_element(ci, b, mask):
 
 # Inputs whose logits reach far beyond those of N(0,1) draws exceed the stated tolerance
 # through the bf16 rounding of the rotated q and k alone (tests/_rounding.py; pinned on the CPU
-# in tests/test_rounding_model.py): there the bound is 1.5 x the rounding model's error on the
+# in tests/test_rounding_model.py): there the bound is 1.25 x the rounding model's error on the
 # same inputs, and the stated tolerance where that is larger.
-MODEL_FACTOR = 1.5
+MODEL_FACTOR = 1.25
 
 
 def _model_bounds(cfg, q, k, v, rows, ref, ref_lse):

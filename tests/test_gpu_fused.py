@@ -14,6 +14,7 @@ import pose_retrieved_kv_b200 as P
 import synth
 from tests._cases import sample_rows
 from tests._gpu import LSE_MAX_ABS, attention_inputs, check_attention, f64, need_gpu
+from tests._rounding import bf16
 
 pytestmark = pytest.mark.gpu
 
@@ -26,6 +27,16 @@ def _rotate(cfg, k, mask=ALL, dyn_flag=None, dyn_src=None, k_rot=None):
     P.prsink_rotate_sinks(P.make_layout(**cfg), kd, kr, mask, dyn_flag, dyn_src)
     assert P.prsink_sync_status() == P.PRSINK_OK
     return kr
+
+
+def _check_rotated(got, ref, what):
+    """The kernel rotates in float32 (cos / sin tables rounded from float64) and rounds once to
+    bf16: it equals the oracle's rotation rounded to bf16 except where the float32 error crosses
+    a rounding boundary, and then by one bf16 unit (or a tiny absolute amount near zero)."""
+    ref16 = bf16(ref)
+    d = np.abs(got - ref16)
+    assert np.mean(d == 0) > 0.99, (what, np.mean(d == 0))
+    assert np.all(d <= 2.0 ** -7 * np.abs(ref16) + 1e-6), (what, d.max())
 
 
 def _rotated_ref(cfg, k):
@@ -47,10 +58,7 @@ def test_rotated_copy_holds_keys_at_their_positions(name, b, mask):
     for slot, (a, e) in enumerate(oracle.slot_ranges(cfg)):
         if slot == cur or not (mask >> slot) & 1:
             continue
-        d = np.abs(kr[:, a:e] - ref[:, a:e])
-        # within one bf16 rounding of the float64 rotation (the kernel rounds once, from fp32)
-        assert np.all(d <= 2.0 ** -8 * np.abs(ref[:, a:e]) + 1e-30), (slot, d.max())
-        assert np.mean(d == 0) > 0.9 or np.mean(d <= 2.0 ** -9 * np.abs(ref[:, a:e])) > 0.99
+        _check_rotated(kr[:, a:e], ref[:, a:e], f"slot {slot}")
 
 
 def test_rotation_mask_and_dynamic_predicates():
@@ -73,7 +81,7 @@ def test_rotation_mask_and_dynamic_predicates():
         a, e = ranges[oracle.SLOT_DYNAMIC]
         assert np.all(np.isnan(kr[:, a:e])) != dyn_written
         if dyn_written:
-            assert np.all(np.abs(kr[:, a:e] - ref[:, a:e]) <= 2.0 ** -8 * np.abs(ref[:, a:e]))
+            _check_rotated(kr[:, a:e], ref[:, a:e], "dynamic")
     kr = f64(_rotate(cfg, k, mask=ALL))
     a, e = ranges[cur]
     # the current slot's rows are only written where they share a tile with rotated slots
