@@ -17,6 +17,12 @@ namespace prsink {
 constexpr int kCopyThreads = 256;
 constexpr int kCopyUnroll = 4;
 
+// Which append kernel runs for head_dim 64 / 128 (the TMA form unless PRSINK_APPEND_TMA=0).
+#ifndef PRSINK_APPEND_TMA
+#define PRSINK_APPEND_TMA 1
+#endif
+static const bool g_append_tma = PRSINK_APPEND_TMA;
+
 // k_new/v_new [n][H][C] 16-byte chunks -> cache [H][T][C] rows start..start+n.
 __global__ void __launch_bounds__(kCopyThreads)
 append_kernel(const uint4* __restrict__ k_new, const uint4* __restrict__ v_new,
@@ -74,6 +80,74 @@ append_rows_kernel(const uint4* __restrict__ k_new, const uint4* __restrict__ v_
     const uint32_t tok = tok0 + u * R;
     if (tok < n) row[static_cast<uint64_t>(tok) * C] = v[u];
   }
+}
+
+// TMA form of the append for head_dim 64 and 128: a unit is the (K|V, head, 128 tokens) tile,
+// loaded token-major from k_new / v_new (box: 64 columns x 1 head x 128 tokens) into shared
+// memory and stored into the slot's rows of the head-major cache (box: 64 columns x 128 rows x 1
+// head; the slot map ends at the slot, so the ragged last tile is clipped).  One thread per CTA
+// keeps kAppendStages tiles in flight: it waits for a stage's load, stores it, and refills the
+// stage once the store has read it.  Waits are bounded (status word on timeout).
+constexpr int kAppendStages = 4;
+constexpr int kAppendTileBytes = 128 * 256;        // one 128-row tile of head_dim 128
+
+struct AppendMaps {
+  CUtensorMap src[2];                              // k_new, v_new   (d, H, n)
+  CUtensorMap dst[2];                              // slot of k_cache, v_cache  (d, n, H)
+};
+
+template <int D>
+__global__ void __launch_bounds__(32, 1)
+append_tma_kernel(const __grid_constant__ AppendMaps maps, int H, int tiles, int* status,
+                  unsigned long long timeout_ns) {
+  extern __shared__ uint8_t dsmem[];
+  __shared__ __align__(8) uint64_t full[kAppendStages];
+  __shared__ AbortState ab;
+  if (threadIdx.x != 0) return;
+  constexpr int kTile = D * 2 * 128;               // bytes of one unit
+  const uint32_t raw = smem_u32(dsmem);
+  const uint32_t sb = (raw + 1023u) & ~1023u;
+  for (int i = 0; i < kAppendStages; ++i) mbar_init(smem_u32(&full[i]), 1);
+  ab.flag = 0;
+  fence_barrier_init();
+  const int per_kv = H * tiles;
+  const int units = 2 * per_kv;
+  auto unit_of = [&](int k) { return static_cast<int>(blockIdx.x) + k * static_cast<int>(gridDim.x); };
+  auto load = [&](int k) {
+    const int u = unit_of(k);
+    const int kv = u / per_kv, r = u - kv * per_kv, h = r / tiles, t = r - h * tiles;
+    const int st = k % kAppendStages;
+    const uint32_t bar = smem_u32(&full[st]);
+    mbar_arrive_expect_tx(bar, kTile);
+    for (int pp = 0; pp < D / 64; ++pp)
+      tma_load_3d(sb + st * kAppendTileBytes + pp * 16384, &maps.src[kv], bar, pp * 64, h,
+                  t * 128);
+  };
+  int n_mine = 0;
+  while (unit_of(n_mine) < units) ++n_mine;
+  for (int k = 0; k < n_mine && k < kAppendStages; ++k) load(k);
+  const uint64_t deadline = globaltimer() + timeout_ns;
+  int k = 0;
+  for (; k < n_mine; ++k) {
+    const int st = k % kAppendStages;
+    if (!mbar_wait(smem_u32(&full[st]), (k / kAppendStages) & 1, &ab, deadline, status)) break;
+    const int u = unit_of(k);
+    const int kv = u / per_kv, r = u - kv * per_kv, h = r / tiles, t = r - h * tiles;
+    for (int pp = 0; pp < D / 64; ++pp)
+      tma_store_3d(&maps.dst[kv], sb + st * kAppendTileBytes + pp * 16384, pp * 64, t * 128, h);
+    bulk_commit();
+    if (k + kAppendStages < n_mine) {
+      bulk_wait_read_all();                        // the store has read the stage
+      load(k + kAppendStages);
+    }
+  }
+  if (ab.flag)                                     // loads still in flight land first
+    for (int j = k; j < n_mine && j < k + kAppendStages; ++j) {
+      const uint64_t dl = globaltimer() + 100000000ull;
+      while (!mbar_try_wait(smem_u32(&full[j % kAppendStages]), (j / kAppendStages) & 1))
+        if (globaltimer() > dl) break;
+    }
+  bulk_wait_all();
 }
 
 // Segment copy: segment y (one (layer, k|v, head) run of `seg_chunks` contiguous chunks) from
@@ -264,7 +338,41 @@ extern "C" int prsink_kv_append(const prsink_layout* layout, const void* k_new,
   auto* vc = static_cast<uint4*>(v_cache);
   const uint64_t start = static_cast<uint64_t>(g.slot_start[dest_slot]);
   constexpr int kU = 4;
-  if (C == 16 || C == 8) {
+  if (g_append_tma && (C == 16 || C == 8)) {
+    AppendMaps maps;
+    const uint64_t H = layout->n_heads, D = layout->head_dim;
+    const uint64_t off = 2ull * D * start;
+    int rc2 = make_map(&maps.src[0], k_new, D, H, n, 2 * D, 2 * D * H, 1, 128);
+    if (!rc2) rc2 = make_map(&maps.src[1], v_new, D, H, n, 2 * D, 2 * D * H, 1, 128);
+    if (!rc2) rc2 = make_map(&maps.dst[0], reinterpret_cast<char*>(k_cache) + off, D, n, H,
+                             2 * D, 2 * D * g.T, 128, 1);
+    if (!rc2) rc2 = make_map(&maps.dst[1], reinterpret_cast<char*>(v_cache) + off, D, n, H,
+                             2 * D, 2 * D * g.T, 128, 1);
+    if (rc2) return rc2;
+    int* sw = status_word_ptr();
+    if (!sw) return PRSINK_ERR_LAUNCH;
+    const int tiles = static_cast<int>((n + 127) / 128);
+    const int units = 2 * layout->n_heads * tiles;
+    int n_sm = 148, dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
+    const int grid = units < n_sm ? units : n_sm;
+    const int smem = kAppendStages * kAppendTileBytes + 1024;
+    static int allowed[64] = {0};
+    if (dev >= 0 && dev < 64 && allowed[dev] < smem) {
+      cudaError_t e = C == 16
+          ? cudaFuncSetAttribute(append_tma_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)
+          : cudaFuncSetAttribute(append_tma_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      if (e != cudaSuccess) return check_launch("prsink_kv_append: shared memory attribute");
+      allowed[dev] = smem;
+    }
+    if (C == 16)
+      append_tma_kernel<128><<<grid, 32, smem, st>>>(maps, layout->n_heads, tiles, sw,
+                                                    2000000000ull);
+    else
+      append_tma_kernel<64><<<grid, 32, smem, st>>>(maps, layout->n_heads, tiles, sw,
+                                                   2000000000ull);
+  } else if (C == 16 || C == 8) {
     const uint32_t rows_per_block = (kCopyThreads / C) * kU;
     dim3 grid(static_cast<unsigned>((n + rows_per_block - 1) / rows_per_block),
               static_cast<unsigned>(layout->n_heads), 2);

@@ -4,6 +4,7 @@
 #pragma once
 
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "../../include/prsink.h"
@@ -26,6 +27,11 @@ struct Geometry {                            // derived token counts of a layout
 int geometry(const prsink_layout* L, Geometry* g);   // validates, PRSINK_OK or ERR_ARG
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// 3-D bf16 TMA tensor map (dims d0 x d1 x d2, strides in bytes for dims 1 and 2) with a
+// 64 x box1 x box2 box, 128-byte swizzle, zero fill out of bounds.  PRSINK_OK or ERR_LAUNCH.
+int make_map(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+             uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box1, uint32_t box2);
 
 // ------------------------------------------------------------------------------------------
 // device side
