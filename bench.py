@@ -666,6 +666,11 @@ def run_kernel_only(args, local_rank: int):
         rec = attention_alone(args.config, args.warmup, args.steps)
         rec["traffic"] = (_profiled_traffic(ATTN_SRC, ATTN_PROFILE)
                           if args.config == "480x480" else None)
+    elif args.only == "split":
+        rec = attention_alone(args.config, args.warmup, args.steps, split=True)
+    elif args.only in ("fused", "rotate"):
+        fused, rot = fused_alone(args.config, args.warmup, args.steps)
+        rec = fused if args.only == "fused" else rot
     elif args.only == "append":
         rec = append_alone(args.config, args.warmup, args.steps)
         rec["traffic"] = (_profiled_traffic(APPEND_SRC, APPEND_PROFILE)
@@ -895,7 +900,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the kernel sub-records and the 300-block stream")
-    ap.add_argument("--only", choices=["attention", "append", "dynfill"], default=None,
+    ap.add_argument("--only", choices=["attention", "append", "dynfill", "fused", "rotate",
+                                       "split"], default=None,
                     help="time one kernel alone at the workload's sizes (for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
