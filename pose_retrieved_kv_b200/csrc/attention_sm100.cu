@@ -599,12 +599,18 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
       };
       int j = 0;
       bool prev_partial = false;
+      int kready0 = 0, kready1 = 0;            // K tiles handed over by the rotation warps
       for (; ok && j < n_live; ++j) {
-        const bool partial = tiles[j] & kTileVfix;        // V touched by the rotation warps
+        const uint16_t te = tiles[j];
+        const bool partial = te & kTileVfix;              // V touched by the rotation warps
         const int st = j & 1;
         // P0(j-1).V(j-1) does not need K(j): issue it before waiting for the rotation
         if (j >= 1 && !pv_mma(0, j - 1, prev_partial)) { ok = false; break; }
-        if (!mbar_wait(bar(B_KREADY + st), (j >> 1) & 1, &ab, deadline, p.status)) { ok = false; break; }
+        // fused form: a tile of the rotated copy goes to the tensor core as it landed
+        const bool direct = kFused && !(te & kTileNew);
+        const uint32_t kbar = direct ? bar(B_KFULL + st) : bar(B_KREADY + st);
+        const uint32_t kpar = direct ? ((j >> 1) & 1) : ((st ? kready1++ : kready0++) & 1);
+        if (!mbar_wait(kbar, kpar, &ab, deadline, p.status)) { ok = false; break; }
         tc_fence_after();
         s_mma(0, st);
         // self-test of the abort path: without this commit the softmax of tile 0 waits until
@@ -657,6 +663,20 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
         const int n = te & kTileIdx;
         const int st = j & 1;
         const uint32_t kt = sK + st * LY::kTileBytes;
+        if (kFused && !(te & kTileNew)) {
+          // a tile of the rotated copy: the MMA reads K as it landed; only the V rows of empty
+          // slots in a boundary tile need zeroing here
+          if (te & kTileVfix) {
+            const int row = n * BN + rt;
+            const bool empty = row < p.T && !((vm >> slot_of(row, p)) & 1u);
+            if (!mbar_wait(bar(B_VFULL + st), (j >> 1) & 1, &ab, deadline, p.status)) break;
+            if (empty)
+              rotate_row<D, RT, RH>(gb + LY::kV + st * LY::kTileBytes, rt, 0, 0, 0, true, tab, p);
+            fence_proxy_async_smem();
+            mbar_arrive(bar(B_VFIX + st));
+          }
+          continue;
+        }
         if (!mbar_wait(bar(B_KFULL + st), (j >> 1) & 1, &ab, deadline, p.status)) break;
         bool empty = false;
         if (kFused && (te & kTileNew)) {
@@ -683,10 +703,6 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
               rotate_row<D, RT, RH>(gb + LY::kK + st * LY::kTileBytes, rt, p.q_frame + ti / p.L_f,
                                     tok / p.grid_w, tok % p.grid_w, false, tab, p);
           }
-        } else if (kFused) {
-          // a tile of the rotated copy: nothing to rotate; find empty-slot rows for V
-          const int row = n * BN + rt;
-          if ((te & kTileVfix) && row < p.T) empty = !((vm >> slot_of(row, p)) & 1u);
         } else {
           const int row = n * BN + rt;
           if (row < p.T) {
