@@ -107,6 +107,7 @@ def _profiled_traffic(src_rel: str, profile_rel: str):
 KERNEL_HEADER = "pose_retrieved_kv_b200/csrc/prsink_internal.cuh"
 ATTN_SRC = "pose_retrieved_kv_b200/csrc/attention_sm100.cu"
 ATTN_PROFILE = "profiles/attention_480x480.md"
+FUSED_PROFILE = "profiles/attention_fused_480x480.md"
 APPEND_SRC = "pose_retrieved_kv_b200/csrc/kv_copy.cu"
 APPEND_PROFILE = "profiles/append_480x480.md"
 
@@ -601,6 +602,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     if rank != 0:
         return None
     peaks = _peaks()
+    prof = FUSED_PROFILE if args.path == "fused" else ATTN_PROFILE
     value = job_throughput(n_layers, args.steps, streams, ms / 1e3)
     flops = 4.0 * lblk * T * d * H                      # QK^T + PV, steady state: all keys valid
     attn_avg_ms = statistics.mean(attn_ms)
@@ -626,10 +628,12 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                       "launches_timed": len(attn_ms), "rank": 0},
         "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
                      "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-                     "traffic": (_profiled_traffic(ATTN_SRC, ATTN_PROFILE)
+                     "traffic": (_profiled_traffic(ATTN_SRC, prof)
                                  if args.config == "480x480" and H == 40 else None),
-                     "traffic_source": f"{ATTN_PROFILE}: ncu dram__bytes_read.sum + "
+                     "traffic_source": f"{prof}: ncu dram__bytes_read.sum + "
                                        "dram__bytes_write.sum, bytes per launch",
+                     "kernel": ("prsink_attention_kernel (fused: the pass's append included)"
+                                if args.path == "fused" else "prsink_attention_kernel"),
                      "peak_source": f"{peaks['source']} bf16_tflops_sustained"},
         "gpu_launches": int(launches),
         "clocks": clk,
@@ -671,6 +675,9 @@ def run_kernel_only(args, local_rank: int):
     elif args.only in ("fused", "rotate"):
         fused, rot = fused_alone(args.config, args.warmup, args.steps)
         rec = fused if args.only == "fused" else rot
+        if args.only == "fused":
+            rec["traffic"] = (_profiled_traffic(ATTN_SRC, FUSED_PROFILE)
+                              if args.config == "480x480" else None)
     elif args.only == "append":
         rec = append_alone(args.config, args.warmup, args.steps)
         rec["traffic"] = (_profiled_traffic(APPEND_SRC, APPEND_PROFILE)
