@@ -91,7 +91,7 @@ enum Bar {
   B_KFULL = 2, B_KREADY = 4, B_KEMPTY = 6,
   B_VFULL = 8, B_VFIX = 10, B_VEMPTY = 12,
   B_SFULL = 14, B_PFULL = 16, B_ODONE = 18,
-  B_FINAL = 20, B_KSTORED = 21, B_COUNT = 22
+  B_FINAL = 20, B_KSTORED = 21, B_COUNT = 23      // B_KSTORED: one per K stage
 };
 
 template <int D>
@@ -465,7 +465,8 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
       mbar_init(bar(B_ODONE + s), 1);
     }
     mbar_init(bar(B_FINAL), 1);
-    mbar_init(bar(B_KSTORED), 1);
+    mbar_init(bar(B_KSTORED + 0), 1);
+    mbar_init(bar(B_KSTORED + 1), 1);
     ab.flag = 0;
     last_k_s = last_v_s = -1;
     unsigned vm = p.valid_mask;
@@ -663,7 +664,10 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
       mbar_arrive(bar(B_QREADY));
       // position of this thread's key row, advanced incrementally from tile to tile
       int cur = -2 * BN, s_cur = 0, frame = 0, y = 0, x = 0;   // no previous row yet
-      int n_stored = 0;                                         // raw K tiles stored so far
+      // raw K tiles stored so far, per stage: a stage is reloaded only after all 128 threads
+      // handed over its previous tile, so the store barrier of a stage never runs two phases
+      // ahead of a thread that still has to see its last phase
+      int n_stored0 = 0, n_stored1 = 0;
       for (int j = 0; j < n_live; ++j) {
         const uint16_t te = tiles[j];
         const int n = te & kTileIdx;
@@ -671,7 +675,10 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
         const uint32_t kt = sK + st * LY::kTileBytes;
         if (kFused && !(te & kTileNew)) {
           // a tile of the rotated copy: the MMA reads K as it landed; only the V rows of empty
-          // slots in a boundary tile need zeroing here
+          // slots in a boundary tile need zeroing here.  The K wait still comes first, for
+          // every tile in order: a parity wait is only sound for a waiter at most one phase
+          // ahead, and skipping tiles would let these warps run further ahead than that.
+          if (!mbar_wait(bar(B_KFULL + st), (j >> 1) & 1, &ab, deadline, p.status)) break;
           if (te & kTileVfix) {
             const int row = n * BN + rt;
             const bool empty = row < p.T && !((vm >> slot_of(row, p)) & 1u);
@@ -694,10 +701,10 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
                 tma_store_3d(&tm_ks, kt + pp * 16384, pp * 64, n * BN, h);
               bulk_commit();
               bulk_wait_read_all();
-              mbar_arrive(bar(B_KSTORED));
+              mbar_arrive(bar(B_KSTORED + st));
             }
-            if (!mbar_wait(bar(B_KSTORED), n_stored & 1, &ab, deadline, p.status)) break;
-            ++n_stored;
+            const int ns = st ? n_stored1++ : n_stored0++;
+            if (!mbar_wait(bar(B_KSTORED + st), ns & 1, &ab, deadline, p.status)) break;
           }
           const int ti = n * BN + rt;
           if (ti < p.L_blk) {

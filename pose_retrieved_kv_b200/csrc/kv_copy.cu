@@ -358,13 +358,15 @@ extern "C" int prsink_kv_append(const prsink_layout* layout, const void* k_new,
     cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
     const int grid = units < n_sm ? units : n_sm;
     const int smem = kAppendStages * kAppendTileBytes + 1024;
-    static int allowed[64] = {0};
-    if (dev >= 0 && dev < 64 && allowed[dev] < smem) {
+    // the attribute belongs to each instantiation: one record per head_dim and device
+    static int allowed[2][64] = {{0}};
+    int& ok = allowed[C == 16 ? 1 : 0][dev >= 0 && dev < 64 ? dev : 0];
+    if (ok < smem) {
       cudaError_t e = C == 16
           ? cudaFuncSetAttribute(append_tma_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)
           : cudaFuncSetAttribute(append_tma_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
       if (e != cudaSuccess) return check_launch("prsink_kv_append: shared memory attribute");
-      allowed[dev] = smem;
+      ok = smem;
     }
     if (C == 16)
       append_tma_kernel<128><<<grid, 32, smem, st>>>(maps, layout->n_heads, tiles, sw,

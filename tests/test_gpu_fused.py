@@ -94,17 +94,20 @@ def test_rotation_mask_and_dynamic_predicates():
 
 
 FUSED_CASES = [("tiny", 7, 0xFF), ("tiny", 1, 0b011011), ("tiny", 2, 0b101111),
-               ("small3d", 11, 0xFF), ("small3d", 4, 0b1010111), ("480x480", 1000, 0xFF),
+               ("small3d", 11, 0xFF), ("small3d", 4, 0b1010111), ("two_tiles", 5, 0xFF),
+               ("two_tiles", 9, 0b1011111), ("480x480", 1000, 0xFF),
                ("480x480", 1, 0b0011011), ("384x672_r4", 1002, 0xFF), ("672x384", 999, 0xFF)]
 SMALL3D = dict(n_heads=3, head_dim=128, grid_h=5, grid_w=7, frames_per_block=3, ref_frames=1,
                ring_slots=3, rope_mode=3, rope_split=(44, 42, 42), rope_base=10000.0)
+# 192 queries: one CTA per head stores both of the block's key tiles (consecutive stores)
+TWO_TILES = dict(SMALL3D, n_heads=2, grid_h=8, grid_w=8)
 
 
 @pytest.mark.parametrize("name,b,mask", FUSED_CASES)
 def test_fused_attention_is_append_then_attention(name, b, mask):
     need_gpu()
-    if name == "small3d":
-        cfg = dict(SMALL3D, block_index=b, valid_mask=mask)
+    if name in ("small3d", "two_tiles"):
+        cfg = dict(SMALL3D if name == "small3d" else TWO_TILES, block_index=b, valid_mask=mask)
     else:
         cfg = synth.preset(name, block_index=b, valid_mask=mask)
     if name in ("480x480", "384x672_r4", "672x384"):
