@@ -114,24 +114,21 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// Softmax exponentials on the FMA pipe for a share of the score columns, so that the
-// special-function unit (16 results per clock per SM, exactly the rate the tensor core produces
-// scores) is not the limit.  Column pair i (0..15) of every 32-column chunk uses the polynomial
-// when bit i of kPolyPairs is set.
+// Softmax exponentials on the FMA pipe for a share of the score columns (column pair i, 0..15,
+// of every 32-column chunk uses the polynomial when bit i of kPolyPairs is set).  Off: measured
+// on a B200 at 480x480, 1/8, 3/16, 1/4 and 1/2 of the exponentials this way were 2-48 % slower,
+// because the one softmax warp per scheduler of a query tile is bound by its own issue and
+// latency, not by the special-function unit.
 #ifndef PRSINK_POLY_PAIRS
-#define PRSINK_POLY_PAIRS 0x8888
+#define PRSINK_POLY_PAIRS 0
 #endif
 constexpr uint32_t kPolyPairs = PRSINK_POLY_PAIRS;
+// Row max with the three-input max.f32 of sm_100 (64 instead of 120 max instructions per row
+// and tile).  Off: measured no faster (fused kernel 2.7 % slower) on a B200.
 #ifndef PRSINK_MAX3
-#define PRSINK_MAX3 1
+#define PRSINK_MAX3 0
 #endif
 constexpr bool kMax3 = PRSINK_MAX3;
-// Read score columns 64..127 from tensor memory a second time after the row max instead of
-// keeping them in registers through the exponentials of columns 0..63.
-#ifndef PRSINK_RELOAD_S
-#define PRSINK_RELOAD_S 0
-#endif
-constexpr bool kReloadS = PRSINK_RELOAD_S;
 
 // 2^x for a pair, by Cody-Waite range reduction (x = n + f, n the nearest integer, taken with the
 // 1.5 * 2^23 rounding constant, f in [-1/2, 1/2]) and a degree-3 polynomial minimising the
@@ -789,12 +786,11 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
       tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
       tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
       tmem_wait_ld();
-      uint32_t mw_s[4] = {~0u, ~0u, ~0u, ~0u};
       if (te & kTileMask) {
         // columns of empty slots and past the end of the cache (or, for the current block's
         // last tile, past its last token): 4 mask words, built per slot
         const int lo = n * BN;
-        uint32_t (&mw)[4] = mw_s;
+        uint32_t mw[4] = {~0u, ~0u, ~0u, ~0u};
         const bool cur_tile = kFused && (te & kTileNew);
         for (int s2 = cur_tile ? p.n_slots : 0; s2 <= p.n_slots; ++s2) {
           int a, e;
@@ -857,23 +853,9 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
       const float2 negm = make_float2(-m, -m);
       float2 sum2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                         make_float2(0.f, 0.f)};               // independent partial sums
-      if constexpr (kReloadS) {
-        // columns 64..127 are read again from tensor memory (the P stores of chunks 0 and 1
-        // overwrite columns 0..31 only), so their registers are free during chunks 0 and 1
-        tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
-        tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
-      }
 #pragma unroll
       for (int ch = 0; ch < 4; ++ch) {
         uint32_t pk[16];
-        if (kReloadS && ch == 2) {
-          tmem_wait_ld();
-          if (te & kTileMask) {           // masked columns again (same words as above)
-#pragma unroll
-            for (int c = 64; c < 128; ++c)
-              if (!((mw_s[c >> 5] >> (c & 31)) & 1u)) s[c] = __float_as_uint(-INFINITY);
-          }
-        }
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const int c = ch * 32 + 2 * i;
