@@ -4,7 +4,9 @@ One step = one block of a 480x480 stream through 40 attention layers (heads 40 x
 fingerprint and pose retrieval with the dynamic-sink fill of every layer, then per layer the 3
 denoising passes and the Clean KV Update pass (KV append into ring slot b mod 3 + PR-Sink
 attention over ref 900 + static 2700 + dynamic 2700 + 3 x 2700 ring = 14400 keys), then the bank
-update.  The bank (M = 5) is filled during the first 20 blocks, which run untimed before the
+update.  By default (``--path fused``) each pass is one prsink_attention_fused launch, which
+stores the pass's K/V into the ring slot itself, after one rotation pass per layer and block
+(prsink_rotate_sinks); ``--path unfused`` launches the append and prsink_attention separately.  The bank (M = 5) is filled during the first 20 blocks, which run untimed before the
 warm-up; the timed blocks are the steady state after it is frozen.
 
 Metric: blocks/s per 40-head layer (layer-blocks per second of the whole job), with the
@@ -173,35 +175,46 @@ class ClockSampler:
 # ------------------------------------------------------------------------------------------
 
 def time_launches(launch, warmup: int, steps: int):
-    """Per-launch device times (ms) of ``launch(i)``: ``warmup`` untimed launches, then
-    ``steps`` launches each between two CUDA events on the current stream.  A device-side sleep
-    is queued ahead of the timed launches so that the host has enqueued them all before the
-    first one starts: each event pair then brackets one kernel's device time, not the host's
-    launch latency."""
+    """Device times (ms) of ``launch(i)`` after ``warmup`` untimed launches: the average launch
+    duration in a steady stream of ``steps`` back-to-back launches (one CUDA event pair around
+    all of them), and each launch's own duration (an event pair per launch, which adds each
+    launch's start-up gap; used for min and max).  A device-side sleep is queued ahead of the
+    timed launches so that the host has enqueued them all before the first one starts."""
     import torch
     for i in range(warmup):
         launch(i)
     torch.cuda.synchronize()
+    torch.cuda._sleep(int(2e6 + 2e5 * steps))
+    b0 = torch.cuda.Event(enable_timing=True)
+    b1 = torch.cuda.Event(enable_timing=True)
+    b0.record()
+    for i in range(steps):
+        launch(warmup + i)
+    b1.record()
+    torch.cuda.synchronize()
+    avg = b0.elapsed_time(b1) / steps
     ev = []
-    torch.cuda._sleep(int(2e6 + 4e5 * steps))        # ~1 ms + ~0.2 ms per launch at 2 GHz
+    torch.cuda._sleep(int(2e6 + 4e5 * steps))
     for i in range(steps):
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record()
-        launch(warmup + i)
+        launch(warmup + steps + i)
         e1.record()
         ev.append((e0, e1))
     torch.cuda.synchronize()
-    return [a.elapsed_time(b) for a, b in ev]
+    return avg, [a.elapsed_time(b) for a, b in ev]
 
 
 def _summary(ms, work, unit, peak, peak_source):
-    avg = statistics.mean(ms)
+    avg, each = ms
     scale = 1e12 if unit == "TFLOP/s" else 1e9
     ach = work / (avg / 1e3) / scale
-    return {"avg_ms": round(avg, 4), "min_ms": round(min(ms), 4), "max_ms": round(max(ms), 4),
-            "launches": len(ms), "achieved": round(ach, 1), "unit": unit, "peak": peak,
-            "frac": round(ach / peak, 4), "peak_source": peak_source}
+    return {"avg_ms": round(avg, 4), "min_ms": round(min(each), 4), "max_ms": round(max(each), 4),
+            "launches": len(each), "achieved": round(ach, 1), "unit": unit, "peak": peak,
+            "frac": round(ach / peak, 4), "peak_source": peak_source,
+            "timing": "avg: back-to-back launches between one event pair; min/max: one event "
+                      "pair per launch"}
 
 
 def attention_alone(name: str, warmup: int, steps: int, repeat: bool = False, nbuf: int = 2,
@@ -891,7 +904,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default="480x480",
                     choices=["480x480", "384x672", "384x672_r4", "672x384", "stream300"])
-    ap.add_argument("--path", choices=["fused", "unfused"], default="unfused",
+    ap.add_argument("--path", choices=["fused", "unfused"], default="fused",
                     help="fused: each pass is one prsink_attention_fused launch (append folded "
                          "in, sinks pre-rotated once per layer and block)")
     ap.add_argument("--partition", choices=["heads", "replicas"], default="heads",
