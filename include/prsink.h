@@ -132,6 +132,26 @@ int prsink_attention_split(const prsink_layout* layout, const void* q, const voi
                            const void* v_cache, void* out, float* lse, const long long* dyn_src,
                            void* scratch, long long scratch_bytes, void* stream);
 
+/* prsink_attention_split without caller scratch, for callers that cannot allocate device
+ * memory: an embedding runtime that owns the device's memory pool and forbids allocations
+ * outside it, or a real-time loop that may not call the allocator (cudaMalloc can synchronise
+ * the device and take milliseconds).  No counterpart on the pages: this is an interface for
+ * such callers, not part of the method.
+ *   The scratch is a file-scope device array of 20 MiB inside the library, held by every GPU
+ *   that loads the library until the process exits: enough for every split plan with
+ *   head_dim <= 128 on a 148-SM device (at most one partial per SM: 19.7 MB); a plan that needs
+ *   more (prsink_attention_scratch_bytes, on a device with more SMs) is rejected with
+ *   PRSINK_ERR_UNSUPPORTED.  The call allocates nothing (no cudaMalloc / cudaFree, no allocating
+ *   library routine); it clears the array's arrival counters on `stream` before the kernel.
+ *   The first call on a device looks up the array's device address with that device current;
+ *   make that first call before any stream capture.  Every call shares the one array, which
+ *   keeps the last call's partial results: calls that overlap on the GPU (other streams, other
+ *   host threads) race on it and must be serialised by the caller.
+ * Arguments, results and other errors as prsink_attention. */
+int prsink_attention_split_noalloc(const prsink_layout* layout, const void* q,
+                                   const void* k_cache, const void* v_cache, void* out,
+                                   float* lse, const long long* dyn_src, void* stream);
+
 /* Scratch bytes prsink_attention_split needs for `layout` on the current device (0 when the
  * last wave is full enough that no split is planned; -1 for an invalid layout). */
 long long prsink_attention_scratch_bytes(const prsink_layout* layout);

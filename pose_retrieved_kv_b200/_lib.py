@@ -105,6 +105,7 @@ def _load():
         "prsink_attention_fused": ([lp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp], i),
         "prsink_attention_split": ([lp, vp, vp, vp, vp, vp, vp, vp, ll, vp], i),
         "prsink_attention_scratch_bytes": ([lp], ll),
+        "prsink_attention_split_noalloc": ([lp, vp, vp, vp, vp, vp, vp, vp], i),
         "prsink_rotate_sinks": ([lp, vp, vp, ctypes.c_uint, vp, vp, vp], i),
         "prsink_retrieve_fallback": ([lp, vp, vp, i, vp, vp, vp, i, ll, vp, vp, vp, vp, vp, vp,
                                       i, vp], i),
@@ -130,7 +131,7 @@ def exported_symbols() -> list:
             "prsink_bank_update", "prsink_sync_status", "prsink_debug_wait_timeout",
             "prsink_retrieve_fallback", "prsink_bank_update_policy", "prsink_attention_fused",
             "prsink_rotate_sinks", "prsink_debug_attention_stall", "prsink_attention_split",
-            "prsink_attention_scratch_bytes"]
+            "prsink_attention_scratch_bytes", "prsink_attention_split_noalloc"]
 
 
 def _check(rc: int, fn: str):
@@ -236,6 +237,21 @@ def prsink_attention_split(layout: Layout, q, k_cache, v_cache, out, scratch, ls
         _ptr(scratch, "scratch", torch.uint8),
         0 if scratch is None else int(scratch.numel()), _stream(stream))
     _check(rc, "prsink_attention_split")
+
+
+def prsink_attention_split_noalloc(layout: Layout, q, k_cache, v_cache, out, lse=None,
+                                   dyn_src=None, stream=None):
+    """prsink_attention_split with the library's static scratch array (no allocation)."""
+    _, lblk, _, T = prsink_layout_tokens(layout)
+    H, d = layout.n_heads, layout.head_dim
+    rc = _lib.prsink_attention_split_noalloc(
+        ctypes.byref(layout), _ptr(q, "q", torch.bfloat16, lblk * H * d),
+        _ptr(k_cache, "k_cache", torch.bfloat16, H * T * d),
+        _ptr(v_cache, "v_cache", torch.bfloat16, H * T * d),
+        _ptr(out, "out", torch.bfloat16, lblk * H * d),
+        _ptr(lse, "lse", torch.float32, H * lblk), _ptr(dyn_src, "dyn_src", torch.int64, 1),
+        _stream(stream))
+    _check(rc, "prsink_attention_split_noalloc")
 
 
 def prsink_attention_fused(layout: Layout, q, k_new, v_new, k_rot, k_cache, v_cache, out,

@@ -1471,6 +1471,68 @@ extern "C" int prsink_attention_split(const prsink_layout* layout, const void* q
                               dyn_src, scratch, scratch_bytes, stream);
 }
 
+// ---- allocation-free form of prsink_attention_split ------------------------------------
+// For callers that cannot allocate device memory: an embedding runtime that owns the device's
+// memory pool and forbids allocations outside it (a framework allocator, a memory-capped
+// serving process), or a real-time loop that may not call the allocator (cudaMalloc can
+// synchronise the device and take milliseconds).  Their scratch is this file-scope device
+// array, so the library allocates nothing when it is used; every GPU that loads the library
+// holds it from module load until the process exits.
+// 20 MiB: a split plan has at most one partial per SM (r units x S shares <= #SM); on a
+// 148-SM device with head_dim 128 that is 148 x 256 rows x (512 + 8) B + counters = 19.7 MB.
+constexpr size_t kStaticSplitScratchBytes = 20ull << 20;
+static __device__ __align__(256) unsigned char g_split_scratch[kStaticSplitScratchBytes];
+
+// Device address of g_split_scratch on the current device.  In host code the symbol's name is
+// only a host-side stand-in, not a device address, so the address is looked up once per device
+// (with that device current) and kept.
+static void* static_split_scratch(const char* what) {
+  static void* addr[64] = {nullptr};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    set_error("%s: no current CUDA device", what);
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lk(mu);
+  if (!addr[dev]) {
+    void* ptr = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&ptr, g_split_scratch);
+    if (e != cudaSuccess || !ptr) {
+      set_error("%s: cudaGetSymbolAddress of the scratch array failed: %s", what,
+                cudaGetErrorString(e));
+      return nullptr;
+    }
+    addr[dev] = ptr;
+  }
+  return addr[dev];
+}
+
+extern "C" int prsink_attention_split_noalloc(const prsink_layout* layout, const void* q,
+                                              const void* k_cache, const void* v_cache,
+                                              void* out, float* lse, const long long* dyn_src,
+                                              void* stream) {
+  using namespace prsink::attn;
+  const char* what = "prsink_attention_split_noalloc";
+  Geometry g;
+  int rc = geometry(layout, &g);
+  if (rc) return rc;
+  const size_t need = plan_split(g, layout->n_heads, layout->head_dim).total();
+  if (need > kStaticSplitScratchBytes) {
+    set_error("%s: this layout needs %zu bytes of split scratch, more than the %zu-byte "
+              "static array; use prsink_attention_split with caller scratch", what, need,
+              kStaticSplitScratchBytes);
+    return PRSINK_ERR_UNSUPPORTED;
+  }
+  void* scratch = nullptr;
+  if (need) {
+    scratch = static_split_scratch(what);
+    if (!scratch) return PRSINK_ERR_LAUNCH;
+  }
+  return attention_split_impl(what, layout, q, k_cache, v_cache, out, lse, dyn_src, scratch,
+                              static_cast<long long>(kStaticSplitScratchBytes), stream);
+}
+
 extern "C" int prsink_attention_fused(const prsink_layout* layout, const void* q,
                                       const void* k_new, const void* v_new, const void* k_rot,
                                       void* k_cache, void* v_cache, void* out, float* lse,
