@@ -90,19 +90,9 @@ enum Bar {
   B_QFULL = 0, B_QREADY = 1,
   B_KFULL = 2, B_KREADY = 4, B_KEMPTY = 6,
   B_VFULL = 8, B_VFIX = 10, B_VEMPTY = 12,
-  B_SFULL = 14, B_PCH = 16,                        // B_PCH: 4 P chunks per query tile
-  B_ODONE = 24, B_FINAL = 26, B_KSTORED = 27,       // B_KSTORED: one per K stage
-  B_COUNT = 29
+  B_SFULL = 14, B_PFULL = 16, B_ODONE = 18,
+  B_FINAL = 20, B_KSTORED = 21, B_COUNT = 23      // B_KSTORED: one per K stage
 };
-
-// P is handed to the P.V MMA in kPChunks pieces (of 128 / kPChunks keys), each on its own
-// barrier, so the tensor core multiplies the first columns of P while the softmax still computes
-// the last ones (the exponentials and P.V of a query tile no longer run one after the other).
-#ifndef PRSINK_P_CHUNKS
-#define PRSINK_P_CHUNKS 4
-#endif
-constexpr int kPChunks = PRSINK_P_CHUNKS;
-static_assert(kPChunks == 1 || kPChunks == 4, "P is handed over whole or in 4 chunks");
 
 template <int D>
 struct Layout {
@@ -468,7 +458,7 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
       mbar_init(bar(B_VFIX + s), 128);
       mbar_init(bar(B_VEMPTY + s), 1);
       mbar_init(bar(B_SFULL + s), 1);
-      for (int c = 0; c < 4; ++c) mbar_init(bar(B_PCH + s * 4 + c), 128);
+      mbar_init(bar(B_PFULL + s), 128);
       mbar_init(bar(B_ODONE + s), 1);
     }
     mbar_init(bar(B_FINAL), 1);
@@ -605,21 +595,10 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
             ++fx;
           }
         }
-        if constexpr (kPChunks == 1) {
-          if (!mbar_wait(bar(B_PCH + qt * 4), i & 1, &ab, deadline, p.status)) return false;
-          tc_fence_after();
-          umma_ts_pv128(tmem + LY::col_o(qt), tmem + LY::col_s(qt), st ? dv1 : dv0,
-                        LY::kIdescPV, i > 0 ? 1u : 0u);
-        } else {
-          // chunk c: keys 32c..32c+31 = P columns 16c.. (bf16 pairs), V steps 2c, 2c+1
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            if (!mbar_wait(bar(B_PCH + qt * 4 + c), i & 1, &ab, deadline, p.status)) return false;
-            tc_fence_after();
-            umma_ts_pv32(tmem + LY::col_o(qt), tmem + LY::col_s(qt) + 16 * c,
-                         (st ? dv1 : dv0) + 256 * c, LY::kIdescPV, (i > 0 || c > 0) ? 1u : 0u);
-          }
-        }
+        if (!mbar_wait(bar(B_PFULL + qt), i & 1, &ab, deadline, p.status)) return false;
+        tc_fence_after();
+        umma_ts_pv128(tmem + LY::col_o(qt), tmem + LY::col_s(qt), st ? dv1 : dv0, LY::kIdescPV,
+                      i > 0 ? 1u : 0u);
         return true;
       };
       int j = 0;
@@ -871,7 +850,7 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
       }
       if (__any_sync(0xffffffffu, rescale)) {   // rows that keep their max scale by alpha = 1
         // O_qt holds every P.V up to tile j-1 (the S(j) commit completed after them); it is
-        // rescaled before any P chunk of tile j is handed over
+        // rescaled before P of tile j is written (measured no slower than after it)
 #pragma unroll 1
         for (int cc = 0; cc < D / 32; ++cc) {
           uint32_t o[32];
@@ -901,12 +880,10 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
           pk[i] = pack_bf16(pr.x, pr.y);
         }
         tmem_st16(tS + ch * 16, pk);
-        if (kPChunks == 4 || ch == 3) {         // hand this chunk (or all of P) over
-          tmem_wait_st();
-          tc_fence_before();
-          mbar_arrive(bar(B_PCH + qt * 4 + (kPChunks == 4 ? ch : 0)));
-        }
       }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(B_PFULL + qt));
       const float2 s01 = fadd2(sum2[0], sum2[1]), s23 = fadd2(sum2[2], sum2[3]);
       const float2 s4 = fadd2(s01, s23);
       l = l * alpha + (s4.x + s4.y);

@@ -320,19 +320,6 @@ __device__ __forceinline__ void umma_ts_pv128(uint32_t d, uint32_t a, uint64_t b
       :: "r"(d), "r"(a), "l"(b), "r"(idesc), "r"(acc) : "memory");
 }
 
-// O (+)= P V over 32 keys (two K = 16 steps) from step `kk0` on: P in TMEM at a + 8*kk, V
-// MN-major at b + 128*kk (descriptor units).  The first step accumulates only if `acc` is set.
-__device__ __forceinline__ void umma_ts_pv32(uint32_t d, uint32_t a, uint64_t b, uint32_t idesc,
-                                             uint32_t acc) {
-  asm volatile(
-      "{\n\t.reg .pred p0, p1;\n\t.reg .b64 b;\n\t.reg .b32 a;\n\t"
-      "setp.ne.b32 p0, %4, 0;\n\tsetp.eq.b32 p1, 0, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p0;\n\t"
-      "add.s32 a, %1, 8;\n\tadd.s64 b, %2, 128;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, p1;\n\t}"
-      :: "r"(d), "r"(a), "l"(b), "r"(idesc), "r"(acc) : "memory");
-}
-
 template <uint32_t N>
 __device__ __forceinline__ void setmaxnreg_inc() {
   asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" :: "n"(N));
