@@ -437,7 +437,9 @@ def _block(st, P, b, kp_dev, ok_dev, qkv, out, events=None, stream=None):
                 e0.record(stream)
             if st.fused:
                 P.prsink_attention_fused(lay, q, kn, vn, st.k_rot[layer], k, v, out, None,
-                                         st.dyn_src)
+                                         st.dyn_src, scratch=st.scratch)
+            elif st.scratch is not None:
+                P.prsink_attention_split(lay, q, k, v, out, st.scratch, None, st.dyn_src)
             else:
                 P.prsink_attention(lay, q, k, v, out, None, st.dyn_src)
             if events is not None:

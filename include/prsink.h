@@ -198,6 +198,17 @@ int prsink_attention_fused(const prsink_layout* layout, const void* q, const voi
                            const void* v_new, const void* k_rot, void* k_cache, void* v_cache,
                            void* out, float* lse, const long long* dyn_src, void* stream);
 
+/* prsink_attention_fused with the last wave split over the key range (as prsink_attention_split;
+ * the scratch size is prsink_attention_scratch_bytes(layout)).  Each tile of the current block is
+ * still stored into the ring slot exactly once, by the share of its unit that attends it.  With
+ * the heads split over several GPUs (5 of 40 heads per GPU at 8 GPUs: 55 units for 148 SMs)
+ * every unit runs as two shares.  Arguments as prsink_attention_fused plus scratch /
+ * scratch_bytes as prsink_attention_split.  Errors: as those two calls. */
+int prsink_attention_fused_split(const prsink_layout* layout, const void* q, const void* k_new,
+                                 const void* v_new, const void* k_rot, void* k_cache,
+                                 void* v_cache, void* out, float* lse, const long long* dyn_src,
+                                 void* scratch, long long scratch_bytes, void* stream);
+
 /* Clean KV Update / per-pass append: write one slot's raw K and V into the caches.
  *
  * [digest] pipeline, inference clause: KV_cache <- KV_cache U Forward(z^0_b, t=0, C) is

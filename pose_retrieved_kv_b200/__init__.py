@@ -14,5 +14,5 @@ from ._lib import (  # noqa: F401
     BANK_MODE_BLEND, BANK_MODE_NONE, BANK_MODE_STORE, BankPolicy, make_policy,
     prsink_bank_update_policy, prsink_retrieve_fallback, prsink_attention_fused,
     prsink_rotate_sinks, prsink_debug_attention_stall, prsink_attention_split,
-    prsink_attention_scratch_bytes, prsink_attention_split_noalloc)
+    prsink_attention_scratch_bytes, prsink_attention_split_noalloc, prsink_attention_fused_split)
 from .stream import PRSinkStream, stream_valid_mask  # noqa: F401

@@ -104,6 +104,7 @@ def _load():
         "prsink_bank_update": ([lp, vp, vp, vp, i, vp, ll, i, vp, vp, vp, i, vp], i),
         "prsink_attention_fused": ([lp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp], i),
         "prsink_attention_split": ([lp, vp, vp, vp, vp, vp, vp, vp, ll, vp], i),
+        "prsink_attention_fused_split": ([lp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ll, vp], i),
         "prsink_attention_scratch_bytes": ([lp], ll),
         "prsink_attention_split_noalloc": ([lp, vp, vp, vp, vp, vp, vp, vp], i),
         "prsink_rotate_sinks": ([lp, vp, vp, ctypes.c_uint, vp, vp, vp], i),
@@ -131,7 +132,8 @@ def exported_symbols() -> list:
             "prsink_bank_update", "prsink_sync_status", "prsink_debug_wait_timeout",
             "prsink_retrieve_fallback", "prsink_bank_update_policy", "prsink_attention_fused",
             "prsink_rotate_sinks", "prsink_debug_attention_stall", "prsink_attention_split",
-            "prsink_attention_scratch_bytes", "prsink_attention_split_noalloc"]
+            "prsink_attention_scratch_bytes", "prsink_attention_split_noalloc",
+            "prsink_attention_fused_split"]
 
 
 def _check(rc: int, fn: str):
@@ -255,9 +257,24 @@ def prsink_attention_split_noalloc(layout: Layout, q, k_cache, v_cache, out, lse
 
 
 def prsink_attention_fused(layout: Layout, q, k_new, v_new, k_rot, k_cache, v_cache, out,
-                           lse=None, dyn_src=None, stream=None):
+                           lse=None, dyn_src=None, stream=None, scratch=None):
+    """With ``scratch`` (a uint8 CUDA tensor of prsink_attention_scratch_bytes bytes) the last
+    wave is split over the key range (prsink_attention_fused_split)."""
     _, lblk, _, T = prsink_layout_tokens(layout)
     H, d = layout.n_heads, layout.head_dim
+    if scratch is not None:
+        rc = _lib.prsink_attention_fused_split(
+            ctypes.byref(layout), _ptr(q, "q", torch.bfloat16, lblk * H * d),
+            _ptr(k_new, "k_new", torch.bfloat16, lblk * H * d),
+            _ptr(v_new, "v_new", torch.bfloat16, lblk * H * d),
+            _ptr(k_rot, "k_rot", torch.bfloat16, H * T * d),
+            _ptr(k_cache, "k_cache", torch.bfloat16, H * T * d),
+            _ptr(v_cache, "v_cache", torch.bfloat16, H * T * d),
+            _ptr(out, "out", torch.bfloat16, lblk * H * d),
+            _ptr(lse, "lse", torch.float32, H * lblk), _ptr(dyn_src, "dyn_src", torch.int64, 1),
+            _ptr(scratch, "scratch", torch.uint8), int(scratch.numel()), _stream(stream))
+        _check(rc, "prsink_attention_fused_split")
+        return
     rc = _lib.prsink_attention_fused(
         ctypes.byref(layout), _ptr(q, "q", torch.bfloat16, lblk * H * d),
         _ptr(k_new, "k_new", torch.bfloat16, lblk * H * d),
@@ -380,3 +397,13 @@ def prsink_debug_wait_timeout(timeout_ns: int, stream=None):
 
 def prsink_debug_attention_stall(timeout_ns: int):
     _check(_lib.prsink_debug_attention_stall(int(timeout_ns)), "prsink_debug_attention_stall")
+
+
+def prsink_attention_fused_split(layout: Layout, q, k_new, v_new, k_rot, k_cache, v_cache, out,
+                                 scratch, lse=None, dyn_src=None, stream=None):
+    """prsink_attention_fused with the last wave split over the key range; ``scratch`` a uint8
+    CUDA tensor of prsink_attention_scratch_bytes(layout) bytes."""
+    if scratch is None:
+        raise ValueError("prsink_attention_fused_split needs scratch")
+    prsink_attention_fused(layout, q, k_new, v_new, k_rot, k_cache, v_cache, out, lse, dyn_src,
+                           stream, scratch=scratch)

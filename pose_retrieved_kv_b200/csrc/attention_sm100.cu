@@ -1534,21 +1534,23 @@ extern "C" int prsink_attention_split_noalloc(const prsink_layout* layout, const
                               static_cast<long long>(kStaticSplitScratchBytes), stream);
 }
 
-extern "C" int prsink_attention_fused(const prsink_layout* layout, const void* q,
-                                      const void* k_new, const void* v_new, const void* k_rot,
-                                      void* k_cache, void* v_cache, void* out, float* lse,
-                                      const long long* dyn_src, void* stream) {
+// Shared by the fused entry points; `scratch` may be null (no split).
+static int attention_fused_impl(const char* what, const prsink_layout* layout, const void* q,
+                                const void* k_new, const void* v_new, const void* k_rot,
+                                void* k_cache, void* v_cache, void* out, float* lse,
+                                const long long* dyn_src, void* scratch, long long scratch_bytes,
+                                bool split, void* stream) {
   using namespace prsink::attn;
   Geometry g;
-  int rc = check_attention_args(layout, &g, "prsink_attention_fused",
-                                {q, k_new, v_new, k_rot, k_cache, v_cache, out}, lse);
+  int rc = check_attention_args(layout, &g, what, {q, k_new, v_new, k_rot, k_cache, v_cache, out},
+                                lse);
   if (rc) return rc;
   if (k_rot == k_cache) {
-    set_error("prsink_attention_fused: k_rot must be a buffer of its own");
+    set_error("%s: k_rot must be a buffer of its own", what);
     return PRSINK_ERR_ARG;
   }
   Params p;
-  rc = fill_params(layout, g, p, "prsink_attention_fused");
+  rc = fill_params(layout, g, p, what);
   if (rc) return rc;
   p.out = static_cast<__nv_bfloat16*>(out);
   p.lse = lse;
@@ -1556,12 +1558,52 @@ extern "C" int prsink_attention_fused(const prsink_layout* layout, const void* q
   p.cur_slot = PRSINK_SLOT_RING0 + static_cast<int>(layout->block_index % layout->ring_slots);
   p.n_cur_tiles = static_cast<int>((g.L_blk + BN - 1) / BN);
   if ((g.T + BN - 1) / BN + p.n_cur_tiles > kMaxTiles) {
-    set_error("prsink_attention_fused: %lld keys exceed the tile limit", g.T);
+    set_error("%s: %lld keys exceed the tile limit", what, g.T);
     return PRSINK_ERR_UNSUPPORTED;
   }
   if (g.L_blk == 0) return PRSINK_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (split) {
+    // a tile of the current block is stored by whichever share of its unit holds it
+    const SplitPlan sp = plan_split(g, layout->n_heads, layout->head_dim);
+    if (sp.n_split > 1) {
+      if (!scratch || (reinterpret_cast<uintptr_t>(scratch) & 255u) ||
+          scratch_bytes < static_cast<long long>(sp.total())) {
+        set_error("%s: scratch must be 256-byte aligned and hold %zu bytes (got %lld)", what,
+                  sp.total(), scratch_bytes);
+        return PRSINK_ERR_ARG;
+      }
+      char* base = static_cast<char*>(scratch);
+      p.part_o = reinterpret_cast<float*>(base);
+      p.part_ml = reinterpret_cast<float2*>(base + sp.o_bytes);
+      p.part_cnt = reinterpret_cast<int*>(base + sp.o_bytes + sp.ml_bytes);
+      p.split_base = sp.split_base;
+      p.n_split = sp.n_split;
+      if (cudaMemsetAsync(p.part_cnt, 0, sp.cnt_bytes, st) != cudaSuccess)
+        return check_launch(what);
+    }
+  }
   const Buffers b{q, k_rot, v_cache, k_new, v_new, k_cache, v_cache};
-  return dispatch<true>(layout, g, b, p, static_cast<cudaStream_t>(stream));
+  return dispatch<true>(layout, g, b, p, st);
+}
+
+extern "C" int prsink_attention_fused(const prsink_layout* layout, const void* q,
+                                      const void* k_new, const void* v_new, const void* k_rot,
+                                      void* k_cache, void* v_cache, void* out, float* lse,
+                                      const long long* dyn_src, void* stream) {
+  return attention_fused_impl("prsink_attention_fused", layout, q, k_new, v_new, k_rot, k_cache,
+                              v_cache, out, lse, dyn_src, nullptr, 0, false, stream);
+}
+
+extern "C" int prsink_attention_fused_split(const prsink_layout* layout, const void* q,
+                                            const void* k_new, const void* v_new,
+                                            const void* k_rot, void* k_cache, void* v_cache,
+                                            void* out, float* lse, const long long* dyn_src,
+                                            void* scratch, long long scratch_bytes,
+                                            void* stream) {
+  return attention_fused_impl("prsink_attention_fused_split", layout, q, k_new, v_new, k_rot,
+                              k_cache, v_cache, out, lse, dyn_src, scratch, scratch_bytes, true,
+                              stream);
 }
 
 extern "C" int prsink_rotate_sinks(const prsink_layout* layout, const void* k_cache,

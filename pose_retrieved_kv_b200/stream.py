@@ -75,6 +75,10 @@ class PRSinkStream:
         self.action = torch.zeros(1, dtype=torch.int32, device=dev)
         self.mode = torch.zeros(1, dtype=torch.int32, device=dev)
         self.frame_ok = torch.ones(3, dtype=torch.uint8, device=dev)
+        # the last wave split over the key range when the device's SMs leave it nearly empty
+        # (few heads per GPU, the 3024-query layouts); scratch for the split partials
+        n = L.prsink_attention_scratch_bytes(lay)
+        self.scratch = torch.empty(n, dtype=torch.uint8, device=dev) if n > 0 else None
         self.fused = bool(fused)
         self.k_rot = (torch.zeros((n_layers, H, self.T, d), dtype=bf, device=dev)
                       if self.fused else None)
@@ -148,7 +152,7 @@ class PRSinkStream:
         if self.fused:
             self.prepare_layer(layer, stream)
             L.prsink_attention_fused(lay, q, k_new, v_new, self.k_rot[layer], k, v, out, lse,
-                                     self.dyn_src, stream)
+                                     self.dyn_src, stream, scratch=self.scratch)
             if clean and self.b == 0:
                 L.prsink_kv_append(lay, k_new, v_new, k, v, L.SLOT_STATIC, stream)
                 self.mark_written(layer, L.SLOT_STATIC)
@@ -156,7 +160,10 @@ class PRSinkStream:
         L.prsink_kv_append(lay, k_new, v_new, k, v, L.SLOT_RING0 + self.b % self.R, stream)
         if clean and self.b == 0:
             L.prsink_kv_append(lay, k_new, v_new, k, v, L.SLOT_STATIC, stream)
-        L.prsink_attention(lay, q, k, v, out, lse, self.dyn_src, stream)
+        if self.scratch is not None:
+            L.prsink_attention_split(lay, q, k, v, out, self.scratch, lse, self.dyn_src, stream)
+        else:
+            L.prsink_attention(lay, q, k, v, out, lse, self.dyn_src, stream)
 
     def end_block(self, stream=None, check: bool = False):
         """Bank update with the clean K/V of block b, then advance to block b+1.  With

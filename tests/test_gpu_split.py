@@ -90,3 +90,39 @@ def test_split_rejects_small_scratch():
     small = torch.empty(n - 256, dtype=torch.uint8, device="cuda")
     with pytest.raises(P.PRSinkError):
         P.prsink_attention_split(lay, q, kv, kv, q.clone(), small)
+
+
+@pytest.mark.parametrize("name,heads,b,mask", [("480x480", 5, 1000, 0xFF),
+                                               ("480x480", 5, 1, 0b0011011),
+                                               ("384x672", 40, 1002, 0xFF)])
+def test_fused_split_is_append_then_attention(name, heads, b, mask):
+    """The fused call with the last wave split: outputs as the oracle's append + attention,
+    the block's raw K/V in its ring slot exactly once (cache bytes bit for bit)."""
+    need_gpu()
+    cfg = synth.preset(name, block_index=b, valid_mask=mask, n_heads=heads)
+    s = oracle.layout_sizes(cfg)
+    H, d = heads, 128
+    q, k, v = attention_inputs(cfg, seed=44)
+    kn = synth.normal_bf16((s["L_blk"], H, d), 44, 7)
+    vn = synth.normal_bf16((s["L_blk"], H, d), 44, 8)
+    lay = P.make_layout(**cfg)
+    kd, vd = k.cuda(), v.cuda()
+    k_rot = torch.empty_like(kd)
+    P.prsink_rotate_sinks(lay, kd, k_rot, 0xFFFF)
+    n = P.prsink_attention_scratch_bytes(lay)
+    assert n > 0
+    scratch = torch.empty(n, dtype=torch.uint8, device="cuda")
+    out = torch.full((s["L_blk"], H, d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lse = torch.full((H, s["L_blk"]), float("nan"), dtype=torch.float32, device="cuda")
+    P.prsink_attention_fused_split(lay, q.cuda(), kn.cuda(), vn.cuda(), k_rot, kd, vd, out,
+                                   scratch, lse)
+    assert P.prsink_sync_status() == P.PRSINK_OK
+    ring = oracle.SLOT_RING0 + b % cfg["ring_slots"]
+    k2, v2 = oracle.kv_append(cfg, f64(kn), f64(vn), f64(k), f64(v), ring)
+    assert np.array_equal(f64(kd), k2) and np.array_equal(f64(vd), v2)
+    rows = sample_rows(s["L_blk"], 13)
+    hs = sorted({0, heads - 2, heads - 1})
+    ref, ref_lse = oracle.attention(dict(cfg, valid_mask=mask | (1 << ring)), f64(q), k2, v2,
+                                    rows=rows, heads=hs)
+    check_attention(f64(out)[rows][:, hs], ref, f"fused split {name}")
+    assert np.abs(f64(lse)[hs][:, rows] - ref_lse).max() <= LSE_MAX_ABS
