@@ -629,9 +629,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "higher_is_better": True, "scaling": "strong" if split else "weak",
         "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (N(0,1) bf16 Q/K/V, clustered synthetic poses; no weights needed)",
-        "config": {"workload": f"per-block step {args.config}: {n_layers} layers x "
-                               f"({PASSES - 1} denoise + 1 clean) x (append + PR-Sink attention), "
-                               "retrieval + dynamic fill, bank update",
+        "config": {"workload": _workload(args.config, n_layers),
                    "path": args.path,
                    "heads": cfg_full["n_heads"], "heads_per_gpu": H, "head_dim": d,
                    "queries": lblk, "keys": T, "ring_slots": cfg["ring_slots"],
@@ -662,6 +660,11 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     if not args.no_cpu_baseline and world == 1:
         res["cpu_baseline"] = cpu_baseline(args, cfg)
     return res
+
+
+def _workload(config: str, n_layers: int) -> str:
+    return (f"per-block step {config}: {n_layers} layers x ({PASSES - 1} denoise + 1 clean) x "
+            "(append + PR-Sink attention), retrieval + dynamic fill, bank update")
 
 
 def _parallelism(args, world):
@@ -877,8 +880,10 @@ def run_reference(args, rank, world):
             "ms_per_step": round(1e3 * wall / args.steps, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (N(0,1) bf16 Q/K/V)",
-            "config": {"workload": f"per-block step {args.config} (oracle, sampled heads)",
-                       "parallelism": "cpu"},
+            "config": {"workload": _workload(args.config, args.layers),
+                       "parallelism": "cpu (float64 oracle, rank 0 only)",
+                       "sampled": f"{heads} of {cfg['n_heads']} heads of one pass per step, "
+                                  "scaled to the layer-block"},
             "cpu_baseline": cb,
             "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
