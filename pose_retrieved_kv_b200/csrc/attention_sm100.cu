@@ -163,20 +163,30 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&b);
 }
 
-__device__ __forceinline__ bool tile_live(int n, unsigned vm, const Params& p) {
-  const int lo = n * BN, hi = min(lo + BN, p.T);
-  for (int s = 0; s < p.n_slots; ++s)
-    if (((vm >> s) & 1u) && p.slot_start[s] < hi && p.slot_start[s + 1] > lo) return true;
-  return false;
-}
-
-__device__ __forceinline__ bool tile_full(int n, unsigned vm, const Params& p) {
-  const int lo = n * BN, hi = lo + BN;
-  if (hi > p.T) return false;
-  for (int s = 0; s < p.n_slots; ++s)
-    if (!((vm >> s) & 1u) && p.slot_start[s] < hi && p.slot_start[s + 1] > lo) return false;
-  return true;
-}
+// Slot bounds held in registers for the tile-list compaction: every bound is read once with a
+// constant index (loops over the slots unrolled to the compile-time maximum), so a warp tests 32
+// tiles with no divergent parameter reads.
+struct SlotBounds {
+  int start[kMaxSlots + 1];
+  __device__ __forceinline__ explicit SlotBounds(const Params& p) {
+#pragma unroll
+    for (int s = 0; s <= kMaxSlots; ++s) start[s] = p.slot_start[s];
+  }
+  // bit 0: tile n holds a key of a slot in vm; bit 1: it also holds rows of a slot not in vm or
+  // rows past the cache end (the tile needs masking)
+  __device__ __forceinline__ int flags(int n, unsigned vm, const Params& p) const {
+    const int lo = n * BN, hi = lo + BN, hil = min(hi, p.T);
+    bool live = false, full = hi <= p.T;
+#pragma unroll
+    for (int s = 0; s < kMaxSlots; ++s) {
+      if (s < p.n_slots) {
+        if ((vm >> s) & 1u) live |= start[s] < hil && start[s + 1] > lo;
+        else full &= !(start[s] < hi && start[s + 1] > lo);
+      }
+    }
+    return (live ? 1 : 0) | (full ? 0 : 2);
+  }
+};
 
 __device__ __forceinline__ int slot_of(int row, const Params& p) {
   int s = 0;
@@ -446,7 +456,8 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
   const int h = unit / p.nqb, qb = unit % p.nqb;
   const int q0 = qb * (NQ * BM);
 
-  if (threadIdx.x == 0) {
+  if (threadIdx.x == 32) {
+    // warp 1: the barriers, then Q, which needs no tile list, goes out at once
     mbar_init(bar(B_QFULL), 1);
     mbar_init(bar(B_QREADY), 128);
     for (int s = 0; s < 2; ++s) {
@@ -465,11 +476,19 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
     mbar_init(bar(B_KSTORED + 1), 1);
     ab.flag = 0;
     last_k_s = last_v_s = -1;
+    fence_barrier_init();
+    mbar_arrive_expect_tx(bar(B_QFULL), NQ * LY::kTileBytes);
+    for (int qt = 0; qt < NQ; ++qt)
+      for (int pp = 0; pp < D / 64; ++pp)
+        tma_load_3d(sQ + qt * LY::kTileBytes + pp * 16384, &tm_q, bar(B_QFULL), pp * 64, h,
+                    q0 + qt * BM);
+  }
+  if (threadIdx.x == 0) {
+    // warp 0: the slots this call attends to, for its tile list below
     unsigned vm = p.valid_mask;
     if (p.dyn_src && *p.dyn_src < 0) vm &= ~(1u << PRSINK_SLOT_DYNAMIC);
     if (kFused) vm &= ~(1u << p.cur_slot);        // its keys come from k_new instead
     vmask_s = vm;
-    fence_barrier_init();
   }
   const int n_tiles = (p.T + BN - 1) / BN;
   if (warp == kProducerWarp && lane == 0) {
@@ -497,14 +516,15 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
     __syncwarp();                                  // vmask_s from lane 0
     // the tiles holding a valid key (boundary tiles flagged for masking), 32 at a time, in order
     const unsigned vm0 = vmask_s;
+    const SlotBounds sbnd(p);
     int base = 0;
     for (int n0 = 0; n0 < n_tiles; n0 += 32) {
       const int n = n0 + lane;
-      const bool live = n < n_tiles && tile_live(n, vm0, p);
-      const uint32_t bal = __ballot_sync(0xffffffffu, live);
-      if (live)
+      const int f = n < n_tiles ? sbnd.flags(n, vm0, p) : 0;
+      const uint32_t bal = __ballot_sync(0xffffffffu, f & 1);
+      if (f & 1)
         tile_list[base + __popc(bal & ((1u << lane) - 1u))] =
-            static_cast<uint16_t>(n | (tile_full(n, vm0, p) ? 0 : (kTileMask | kTileVfix)));
+            static_cast<uint16_t>(n | ((f & 2) ? (kTileMask | kTileVfix) : 0));
       base += __popc(bal);
     }
     if (kFused) {
@@ -559,16 +579,10 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
     last_v_s = j;
     return true;
   };
-  // the producer sends Q and the first two K/V tiles out at once (their stages are free, so
-  // nothing waits)
-  if (warp == kProducerWarp && lane == 0) {
-    mbar_arrive_expect_tx(bar(B_QFULL), NQ * LY::kTileBytes);
-    for (int qt = 0; qt < NQ; ++qt)
-      for (int pp = 0; pp < D / 64; ++pp)
-        tma_load_3d(sQ + qt * LY::kTileBytes + pp * 16384, &tm_q, bar(B_QFULL), pp * 64, h,
-                    q0 + qt * BM);
+  // the producer sends the first two K/V tiles out at once (their stages are free, so nothing
+  // waits)
+  if (warp == kProducerWarp && lane == 0)
     for (int j = 0; j < 2 && j < n_live; ++j) load_kv(j);
-  }
   if constexpr (kFused) {
     build_rope_tables<D, RT, RH>(gb + LY::kTab, p, threadIdx.x, kThreads);
     __syncthreads();
@@ -578,7 +592,7 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
     setmaxnreg_dec<80>();
     if (warp == kProducerWarp && lane == 0) {
       // ---------------------------------------------------------------- TMA producer
-      // (Q and tiles 0, 1 went out before the tables)
+      // (Q and tiles 0, 1 are already on their way)
       for (int j = 2; j < n_live; ++j)
         if (!load_kv(j)) break;
     } else if (warp == kMmaWarp && lane == 0) {
@@ -1068,10 +1082,12 @@ prsink_rotate_kernel(const __grid_constant__ CUtensorMap tm_src,
   if (warp == 0) {
     __syncwarp();                                  // mask_s from lane 0
     const int n_tiles = (p.T + BN - 1) / BN;
+    const unsigned m = mask_s;
+    const SlotBounds sbnd(p);
     int base = 0;
     for (int n0 = 0; n0 < n_tiles; n0 += 32) {
       const int n = n0 + lane;
-      const bool live = n < n_tiles && tile_live(n, mask_s, p);
+      const bool live = n < n_tiles && (sbnd.flags(n, m, p) & 1);
       const uint32_t bal = __ballot_sync(0xffffffffu, live);
       if (live) tile_list[base + __popc(bal & ((1u << lane) - 1u))] = static_cast<uint16_t>(n);
       base += __popc(bal);
