@@ -7,13 +7,15 @@
 // Warp roles (512 threads; setmaxnreg gives the softmax warps 184 registers, the rotation
 // warps 64 and the producer / MMA warps 80):
 //   warps 0-3   softmax of Q0, warps 4-7 softmax of Q1: thread t owns query row t (TMEM lane
-//               t); it reads S from TMEM, keeps the running max and sum, writes P as bf16 back
-//               into the S columns (the A operand of the P.V MMA), rescales O in TMEM when the
-//               max grew by more than 2^8, and finally normalises and stores O;
-//   warps 8-11  rotation: rotate Q0/Q1 once and every K tile in place at the keys' current
-//               logical positions (interleaved RoFormer pairs, per-axis cos/sin tables in
-//               shared memory); zero the K and V rows of empty slots in boundary tiles;
-//   warp  12    TMA producer: Q once, then K and V tiles, each through its own 2-stage ring;
+//               t); it first rotates its own row of Q in shared memory, then reads S from
+//               TMEM, keeps the running max and sum, writes P as bf16 back into the S columns
+//               (the A operand of the P.V MMA), rescales O in TMEM when the max grew by more
+//               than 2^8, and finally normalises and stores O;
+//   warps 8-11  rotation: rotate every K tile in place at the keys' current logical positions
+//               (interleaved RoFormer pairs, per-axis cos/sin tables in shared memory); zero
+//               the K and V rows of empty slots in boundary tiles;
+//   warp  12    TMA producer: K and V tiles, each through its own 2-stage ring (Q is sent by
+//               warp 1 as soon as the barriers exist);
 //   warp  13    MMA issuer: per key tile j, P0(j-1).V, S0(j) = Q0 K^T, P1(j-1).V, S1(j).
 // Key tiles run over the physical rows of the cache: softmax attention does not depend on the
 // order of the keys, only on their positions, so each key is rotated at the position of its
@@ -459,7 +461,7 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
   if (threadIdx.x == 32) {
     // warp 1: the barriers, then Q, which needs no tile list, goes out at once
     mbar_init(bar(B_QFULL), 1);
-    mbar_init(bar(B_QREADY), 128);
+    mbar_init(bar(B_QREADY), NQ * BM);
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar(B_KFULL + s), 1);
       mbar_init(bar(B_KREADY + s), 128);
@@ -668,22 +670,7 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
     // ------------------------------------------------------------------ rotation
     setmaxnreg_dec<64>();
     const int rt = threadIdx.x - kRotWarp0 * 32;          // row of the tile, 0..127
-    if (mbar_wait(bar(B_QFULL), 0, &ab, deadline, p.status)) {
-      for (int qt = 0; qt < NQ; ++qt) {
-        const int qi = q0 + qt * BM + rt;
-        if (qi < p.L_blk) {
-          const int tok = qi % p.L_f;
-          if constexpr (RT > 0)
-            rotate_row_grouped<RT, RH>(sQ + qt * LY::kTileBytes, rt, p.q_frame + qi / p.L_f,
-                                       tok / p.grid_w, tok % p.grid_w, false, smem_u32(gcs),
-                                       smem_u32(gns), p);
-          else
-            rotate_row<D, RT, RH>(gb + LY::kQ + qt * LY::kTileBytes, rt, p.q_frame + qi / p.L_f,
-                                  tok / p.grid_w, tok % p.grid_w, false, tab, p);
-        }
-      }
-      fence_proxy_async_smem();
-      mbar_arrive(bar(B_QREADY));
+    {   // (Q is rotated by the softmax warps, one query row per thread)
       // position of this thread's key row, advanced incrementally from tile to tile
       int cur = -2 * BN, s_cur = 0, frame = 0, y = 0, x = 0;   // no previous row yet
       // raw K tiles stored so far, per stage: a stage is reloaded only after all 128 threads
@@ -798,8 +785,25 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
     const float2 scale2 = make_float2(p.scale_log2, p.scale_log2);
     float m = -INFINITY, l = 0.f;
     int j = 0;
-    bool ok = true;
-    for (; j < n_live; ++j) {
+    // this thread's own query row, rotated at its position while the rotation warps take the
+    // first key tiles
+    bool ok = __all_sync(0xffffffffu, mbar_wait(bar(B_QFULL), 0, &ab, deadline, p.status));
+    if (ok) {
+      const int qi = q0 + qt * BM + t;
+      if (qi < p.L_blk) {
+        const int tok = qi % p.L_f;
+        if constexpr (RT > 0)
+          rotate_row_grouped<RT, RH>(sQ + qt * LY::kTileBytes, t, p.q_frame + qi / p.L_f,
+                                     tok / p.grid_w, tok % p.grid_w, false, smem_u32(gcs),
+                                     smem_u32(gns), p);
+        else
+          rotate_row<D, RT, RH>(gb + LY::kQ + qt * LY::kTileBytes, t, p.q_frame + qi / p.L_f,
+                                tok / p.grid_w, tok % p.grid_w, false, tab, p);
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(bar(B_QREADY));
+    }
+    for (; ok && j < n_live; ++j) {
       const uint16_t te = tiles[j];
       const int n = te & kTileIdx;
       ok = mbar_wait(bar(B_SFULL + qt), j & 1, &ab, deadline, p.status);
