@@ -149,7 +149,7 @@ class ClockSampler:
             self.proc.wait(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
-        sm, smax, reasons = [], 0.0, set()
+        sm, pw, smax, reasons = [], [], 0.0, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for ln in self.lines:
             parts = [p.strip() for p in ln.split(",")]
@@ -160,14 +160,21 @@ class ClockSampler:
                 smax = max(smax, float(parts[2]))
             except ValueError:
                 continue
+            try:
+                pw.append(float(parts[3]))
+            except ValueError:
+                pass
             for nm, val in zip(names, parts[5:9]):
                 if val.lower() == "active":
                     reasons.add(nm)
         if not sm:
             return None
         loaded = [v for v in sm if v > 0.5 * smax] or sm
-        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": smax,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        rec = {"sm_mhz": statistics.median(loaded), "sm_max_mhz": smax,
+               "reasons": sorted(reasons), "samples": len(sm)}
+        if pw:
+            rec["power_w"] = statistics.median(pw)    # board power draw, median of the samples
+        return rec
 
 
 # ------------------------------------------------------------------------------------------
