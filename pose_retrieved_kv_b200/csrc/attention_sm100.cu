@@ -427,7 +427,8 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
                         const __grid_constant__ CUtensorMap tm_kn,
                         const __grid_constant__ CUtensorMap tm_vn,
                         const __grid_constant__ CUtensorMap tm_ks,
-                        const __grid_constant__ CUtensorMap tm_vs, const Params p) {
+                        const __grid_constant__ CUtensorMap tm_vs,
+                        const __grid_constant__ CUtensorMap tm_o, const Params p) {
   using LY = Layout<D>;
   extern __shared__ uint8_t dsmem[];
   __shared__ __align__(8) uint64_t bars[B_COUNT];
@@ -917,7 +918,10 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
       const float2 s4 = fadd2(s01, s23);
       l = l * alpha + (s4.x + s4.y);
     }
-    // epilogue: O / l -> bf16, one 2*D-byte row per thread
+    // epilogue: O / l -> bf16.  A whole unit stages its rows in the tile's own Q buffer (free:
+    // ODONE follows every S MMA), in the layout the Q load used (128-byte swizzled panels of 64
+    // columns), and one thread stores the tile with TMA (rows past the block are clipped); a
+    // split CTA writes its unnormalised float32 partial row (O, max, sum) for the combine.
     const int qi = q0 + qt * BM + t;
     float inv = 0.f;
     bool have = false;
@@ -927,8 +931,7 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
       tc_fence_after();
       inv = l > 0.f ? 1.f / l : 0.f;
     }
-    __nv_bfloat16* orow = p.out + (static_cast<size_t>(qi) * p.H + h) * D;
-    // a split CTA writes its unnormalised partial (O, max, sum) for the combine instead
+    const uint32_t so = sQ + qt * LY::kTileBytes;
     const size_t slot = static_cast<size_t>(unit - p.split_base) * n_split + split;
     float* prow = n_split > 1 ? p.part_o + (slot * (NQ * BM) + qt * BM + t) * D : nullptr;
     if (n_split > 1)
@@ -949,7 +952,7 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
         for (int i = 0; i < 32; i += 4)
           *reinterpret_cast<uint4*>(prow + cc * 32 + i) = make_uint4(o[i], o[i + 1], o[i + 2],
                                                                      o[i + 3]);
-      } else if (qi < p.L_blk) {
+      } else {
 #pragma unroll
         for (int i = 0; i < 32; i += 8) {
           uint4 v;
@@ -957,8 +960,19 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
           v.y = pack_bf16(__uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
           v.z = pack_bf16(__uint_as_float(o[i + 4]) * inv, __uint_as_float(o[i + 5]) * inv);
           v.w = pack_bf16(__uint_as_float(o[i + 6]) * inv, __uint_as_float(o[i + 7]) * inv);
-          *reinterpret_cast<uint4*>(orow + cc * 32 + i) = v;
+          const int k = (cc * 32 + i) >> 3;           // 16-byte chunk of the row
+          sts_u4(so + (k >> 3) * 16384 + t * 128 + (((k & 7) ^ (t & 7)) << 4), v);
         }
+      }
+    }
+    if (!prow) {
+      fence_proxy_async_smem();
+      named_bar_sync(1 + qt, BM);                     // the tile's 128 rows are staged
+      if (t == 0) {
+        for (int pp = 0; pp < D / 64; ++pp)
+          tma_store_3d(&tm_o, so + pp * 16384, pp * 64, h, q0 + qt * BM);
+        bulk_commit();
+        bulk_wait_all();                              // complete before the CTA exits
       }
     }
     if (p.lse && qi < p.L_blk && n_split == 1)
@@ -1211,8 +1225,10 @@ static int launch(const prsink_layout* L, const Geometry& g, const Buffers& b, P
                   cudaStream_t st) {
   const char* what = kFused ? "prsink_attention_fused" : "prsink_attention";
   const uint64_t H = L->n_heads;
-  CUtensorMap mq, mk, mv, mkn, mvn, mks, mvs;
+  CUtensorMap mq, mk, mv, mkn, mvn, mks, mvs, mo;
   int rc = make_map(&mq, b.q, D, H, g.L_blk, 2ull * D, 2ull * D * H, 1, BM);
+  // the output has Q's layout ([L_blk][H][d]); whole tiles leave through TMA stores
+  if (!rc) rc = make_map(&mo, p.out, D, H, g.L_blk, 2ull * D, 2ull * D * H, 1, BM);
   if (!rc) rc = make_map(&mk, b.k, D, g.T, H, 2ull * D, 2ull * D * g.T, BN, 1);
   if (!rc) rc = make_map(&mv, b.v, D, g.T, H, 2ull * D, 2ull * D * g.T, BN, 1);
   if (kFused) {
@@ -1242,7 +1258,7 @@ static int launch(const prsink_layout* L, const Geometry& g, const Buffers& b, P
   const int units = p.nqb * L->n_heads;
   const int ctas = p.split_base + (units - p.split_base) * p.n_split;
   prsink_attention_kernel<D, RT, RH, kFused><<<ctas, kThreads, smem, st>>>(mq, mk, mv, mkn, mvn,
-                                                                          mks, mvs, p);
+                                                                          mks, mvs, mo, p);
   count_launch();
   return check_launch(what);
 }

@@ -102,6 +102,12 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, AbortSt
   return true;
 }
 
+// bar.sync on named barrier `id` (1..15) for `count` threads (a multiple of 32): a barrier for
+// a subset of the CTA's warps
+__device__ __forceinline__ void named_bar_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 __device__ __forceinline__ void fence_barrier_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
