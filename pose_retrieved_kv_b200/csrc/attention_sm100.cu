@@ -1063,11 +1063,14 @@ prsink_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
 // prsink_rotate_sinks: the raw keys of the slots in the rotation mask rotated at this block's
 // positions into k_rot (same [H][T][d] layout), with the attention kernel's own rotation code,
 // so that the fused attention reads keys bitwise equal to the ones it would rotate itself.
-// Work item = (head, key tile of 128 rows); a CTA streams its items through two shared-memory
-// stages: TMA load of the raw tile, one row per thread rotated in place, TMA store.  Rows of
-// other slots that share a boundary tile are rotated and stored too: their rotated copies are
-// either rewritten identically (slots whose positions are fixed) or never read.
-constexpr int kRotThreads = 128;
+// Work item = (head, key tile of 128 rows).  A CTA (one per SM) runs kRotGroups independent
+// 128-thread pipelines that share one copy of the RoPE tables; each streams its items through
+// its own two shared-memory stages: TMA load of the raw tile, one row per thread rotated in
+// place, TMA store.  Rows of other slots that share a boundary tile are rotated and stored too:
+// their rotated copies are either rewritten identically (slots whose positions are fixed) or
+// never read.
+constexpr int kRotGroups = 3;
+constexpr int kRotThreads = 128 * kRotGroups;
 
 template <int D, int RT, int RH>
 __global__ void __launch_bounds__(kRotThreads)
@@ -1075,20 +1078,24 @@ prsink_rotate_kernel(const __grid_constant__ CUtensorMap tm_src,
                      const __grid_constant__ CUtensorMap tm_dst, const Params p) {
   using LY = Layout<D>;
   extern __shared__ uint8_t dsmem[];
-  __shared__ __align__(8) uint64_t full[2];
+  __shared__ __align__(8) uint64_t full[kRotGroups][2];
   __shared__ AbortState ab;
   __shared__ unsigned mask_s;
   __shared__ uint16_t tile_list[kMaxTiles];
   __shared__ int n_live_s;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int rt = threadIdx.x;
+  const int grp = threadIdx.x >> 7, rt = threadIdx.x & 127;   // pipeline, row of the tile
+  const bool leader = rt == 0;
   const uint32_t raw = smem_u32(dsmem);
   const uint32_t sb = (raw + 1023u) & ~1023u;
   uint8_t* gb = dsmem + (sb - raw);
-  constexpr int kTabOff = 2 * LY::kTileBytes;
+  const uint32_t stage0 = sb + grp * 2 * LY::kTileBytes;      // this pipeline's two stages
+  constexpr int kTabOff = kRotGroups * 2 * LY::kTileBytes;
   if (threadIdx.x == 0) {
-    mbar_init(smem_u32(&full[0]), 1);
-    mbar_init(smem_u32(&full[1]), 1);
+    for (int g = 0; g < kRotGroups; ++g) {
+      mbar_init(smem_u32(&full[g][0]), 1);
+      mbar_init(smem_u32(&full[g][1]), 1);
+    }
     ab.flag = 0;
     unsigned m = p.rot_mask & p.valid_mask;
     if (p.cur_slot >= 0) m &= ~(1u << p.cur_slot);
@@ -1115,22 +1122,24 @@ prsink_rotate_kernel(const __grid_constant__ CUtensorMap tm_src,
   __syncthreads();
   const int n_live = n_live_s;
   const int total = n_live * p.H;
+  const int stride = gridDim.x * kRotGroups;
+  const int w0 = blockIdx.x * kRotGroups + grp;
   const uint64_t deadline = globaltimer() + p.timeout_ns;
   auto item = [&](int w, int& n, int& h) { h = w / n_live; n = tile_list[w - h * n_live]; };
   auto load = [&](int w, int st) {
     int n, h;
     item(w, n, h);
-    const uint32_t bar = smem_u32(&full[st]);
+    const uint32_t bar = smem_u32(&full[grp][st]);
     mbar_arrive_expect_tx(bar, LY::kTileBytes);
     for (int pp = 0; pp < D / 64; ++pp)
-      tma_load_3d(sb + st * LY::kTileBytes + pp * 16384, &tm_src, bar, pp * 64, n * BN, h);
+      tma_load_3d(stage0 + st * LY::kTileBytes + pp * 16384, &tm_src, bar, pp * 64, n * BN, h);
   };
-  // the first item's load goes out before the RoPE tables are built
+  // each pipeline's first load goes out before the RoPE tables are built
   int i = 0, last_load = -1;
-  if (threadIdx.x == 0 && static_cast<int>(blockIdx.x) < total) {
+  if (leader && w0 < total) {
     prefetch_tmap(&tm_src);
     prefetch_tmap(&tm_dst);
-    load(blockIdx.x, 0);
+    load(w0, 0);
     last_load = 0;
   }
   float4* gcs = reinterpret_cast<float4*>(gb + kTabOff);
@@ -1140,18 +1149,18 @@ prsink_rotate_kernel(const __grid_constant__ CUtensorMap tm_src,
   float2* tab = reinterpret_cast<float2*>(gb + kTabOff);
   build_rope_tables<D, RT, RH>(gb + kTabOff, p, threadIdx.x, kRotThreads);
   __syncthreads();
-  for (int w = blockIdx.x; w < total; w += gridDim.x, ++i) {
+  for (int w = w0; w < total; w += stride, ++i) {
     const int st = i & 1;
-    const int wn = w + gridDim.x;
-    if (threadIdx.x == 0 && wn < total) {
+    const int wn = w + stride;
+    if (leader && wn < total) {
       bulk_wait_read_all();             // the store of item i-1 has read stage st^1
       load(wn, st ^ 1);
       last_load = i + 1;
     }
-    // every thread takes the same decision (a wait that gave up in one thread ends the loop
-    // for all, so no thread is left behind at the barrier below)
-    if (!__syncthreads_and(mbar_wait(smem_u32(&full[st]), (i >> 1) & 1, &ab, deadline,
-                                     p.status)))
+    // every thread of the pipeline takes the same decision (a wait that gave up in one thread
+    // ends the loop for all, so no thread is left behind at the barrier below)
+    if (!named_bar_and(1 + grp, 128, mbar_wait(smem_u32(&full[grp][st]), (i >> 1) & 1, &ab,
+                                                deadline, p.status)))
       break;
     int n, h;
     item(w, n, h);
@@ -1162,24 +1171,24 @@ prsink_rotate_kernel(const __grid_constant__ CUtensorMap tm_src,
       const int tok = u % p.L_f;
       const int frame = p.slot_frame[s] + u / p.L_f;
       if constexpr (RT > 0)
-        rotate_row_grouped<RT, RH>(sb + st * LY::kTileBytes, rt, frame, tok / p.grid_w,
+        rotate_row_grouped<RT, RH>(stage0 + st * LY::kTileBytes, rt, frame, tok / p.grid_w,
                                    tok % p.grid_w, false, smem_u32(gcs), smem_u32(gns), p);
       else
-        rotate_row<D, RT, RH>(gb + st * LY::kTileBytes, rt, frame, tok / p.grid_w,
-                              tok % p.grid_w, false, tab, p);
+        rotate_row<D, RT, RH>(gb + (stage0 - sb) + st * LY::kTileBytes, rt, frame,
+                              tok / p.grid_w, tok % p.grid_w, false, tab, p);
     }
     fence_proxy_async_smem();
-    __syncthreads();
-    if (threadIdx.x == 0) {
+    named_bar_sync(1 + grp, 128);
+    if (leader) {
       for (int pp = 0; pp < D / 64; ++pp)
-        tma_store_3d(&tm_dst, sb + st * LY::kTileBytes + pp * 16384, pp * 64, n * BN, h);
+        tma_store_3d(&tm_dst, stage0 + st * LY::kTileBytes + pp * 16384, pp * 64, n * BN, h);
       bulk_commit();
     }
   }
-  if (threadIdx.x == 0) {
+  if (leader) {
     if (ab.flag) {                      // let loads in flight land before shared memory goes
       for (int k = last_load - 1; k <= last_load; ++k)
-        if (k >= i) drain_wait(smem_u32(&full[k & 1]), (k >> 1) & 1, 100000000ull);
+        if (k >= i) drain_wait(smem_u32(&full[grp][k & 1]), (k >> 1) & 1, 100000000ull);
     }
     bulk_wait_all();
   }
@@ -1277,16 +1286,18 @@ static int launch_rotate(const prsink_layout* L, const Geometry& g, const void* 
               kTableMaxBytes);
     return PRSINK_ERR_UNSUPPORTED;
   }
-  const int smem = 2 * Layout<D>::kTileBytes + tab + 1024;
+  const int smem = kRotGroups * 2 * Layout<D>::kTileBytes + tab + 1024;
   static int allowed[64] = {0};
   rc = allow_smem(prsink_rotate_kernel<D, RT, RH>, smem, allowed, "prsink_rotate_sinks");
   if (rc) return rc;
   int n_sm = 148, dev = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
-  // work items: every (head, key tile); two CTAs per SM stream them
+  // work items: the (head, key tile) pairs of the rotated slots; one CTA per SM, kRotGroups
+  // pipelines each, stream them
   const long long items = static_cast<long long>(H) * ((g.T + BN - 1) / BN);
-  const int grid = static_cast<int>(items < 2ll * n_sm ? items : 2ll * n_sm);
+  const long long ctas = (items + kRotGroups - 1) / kRotGroups;
+  const int grid = static_cast<int>(ctas < n_sm ? ctas : n_sm);
   prsink_rotate_kernel<D, RT, RH><<<grid, kRotThreads, smem, st>>>(ms, md, p);
   count_launch();
   return check_launch("prsink_rotate_sinks");
