@@ -86,9 +86,10 @@ append_rows_kernel(const uint4* __restrict__ k_new, const uint4* __restrict__ v_
 // loaded token-major from k_new / v_new (box: 64 columns x 1 head x 128 tokens) into shared
 // memory and stored into the slot's rows of the head-major cache (box: 64 columns x 128 rows x 1
 // head; the slot map ends at the slot, so the ragged last tile is clipped).  One thread per CTA
-// keeps kAppendStages tiles in flight: it waits for a stage's load, stores it, and refills the
-// stage once the store has read it.  Waits are bounded (status word on timeout).
-constexpr int kAppendStages = 4;
+// keeps the stages busy: it waits for a stage's load and stores it, then refills the stage of
+// the PREVIOUS tile once that older store has read it, so a store never waits for itself and
+// kAppendStages - 1 loads stay in flight.  Waits are bounded (status word on timeout).
+constexpr int kAppendStages = 6;
 constexpr int kAppendTileBytes = 128 * 256;        // one 128-row tile of head_dim 128
 
 struct AppendMaps {
@@ -125,7 +126,11 @@ append_tma_kernel(const __grid_constant__ AppendMaps maps, int H, int tiles, int
   };
   int n_mine = 0;
   while (unit_of(n_mine) < units) ++n_mine;
-  for (int k = 0; k < n_mine && k < kAppendStages; ++k) load(k);
+  int last_load = -1;                              // highest tile whose load went out
+  for (int k = 0; k < n_mine && k < kAppendStages; ++k) {
+    load(k);
+    last_load = k;
+  }
   const uint64_t deadline = globaltimer() + timeout_ns;
   int k = 0;
   for (; k < n_mine; ++k) {
@@ -136,13 +141,14 @@ append_tma_kernel(const __grid_constant__ AppendMaps maps, int H, int tiles, int
     for (int pp = 0; pp < D / 64; ++pp)
       tma_store_3d(&maps.dst[kv], sb + st * kAppendTileBytes + pp * 16384, pp * 64, t * 128, h);
     bulk_commit();
-    if (k + kAppendStages < n_mine) {
-      bulk_wait_read_all();                        // the store has read the stage
-      load(k + kAppendStages);
+    if (k >= 1 && k - 1 + kAppendStages < n_mine) {
+      bulk_wait_read_all_but_newest();             // the store of tile k-1 has read its stage
+      load(k - 1 + kAppendStages);
+      last_load = k - 1 + kAppendStages;
     }
   }
   if (ab.flag)                                     // loads still in flight land first
-    for (int j = k; j < n_mine && j < k + kAppendStages; ++j) {
+    for (int j = k; j <= last_load; ++j) {
       const uint64_t dl = globaltimer() + 100000000ull;
       while (!mbar_try_wait(smem_u32(&full[j % kAppendStages]), (j / kAppendStages) & 1))
         if (globaltimer() > dl) break;
