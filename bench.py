@@ -264,10 +264,11 @@ def attention_alone(name: str, warmup: int, steps: int, repeat: bool = False, nb
     return rec
 
 
-def fused_alone(name: str, warmup: int, steps: int):
+def fused_alone(name: str, warmup: int, steps: int, split: bool = False):
     """prsink_attention_fused (append folded in, sinks read pre-rotated) and the rotation pass
     prsink_rotate_sinks, each timed alone at a workload's full size on two alternating input
-    sets (each larger than L2)."""
+    sets (each larger than L2).  ``split``: the last wave split over the key range, as the
+    stream runs it when the plan calls for it (prsink_attention_fused_split)."""
     import torch
 
     import pose_retrieved_kv_b200 as P
@@ -287,10 +288,13 @@ def fused_alone(name: str, warmup: int, steps: int):
                          kn=synth.normal_bf16((lblk, H, d), 5 + i, 3).cuda(),
                          vn=synth.normal_bf16((lblk, H, d), 5 + i, 4).cuda()))
     out = torch.empty((lblk, H, d), dtype=torch.bfloat16, device="cuda")
+    n_scr = P.prsink_attention_scratch_bytes(lay) if split else 0
+    scratch = torch.empty(n_scr, dtype=torch.uint8, device="cuda") if n_scr > 0 else None
 
     def fused(i):
         x = sets[i % 2]
-        P.prsink_attention_fused(lay, x["q"], x["kn"], x["vn"], x["kr"], x["k"], x["v"], out)
+        P.prsink_attention_fused(lay, x["q"], x["kn"], x["vn"], x["kr"], x["k"], x["v"], out,
+                                 scratch=scratch)
 
     ring = ((1 << cfg["ring_slots"]) - 1) << P.SLOT_RING0
 
@@ -308,8 +312,9 @@ def fused_alone(name: str, warmup: int, steps: int):
     n_rot = (cfg["ring_slots"] - 1) * lblk * H             # the two older ring slots
     rot = _summary(ms_r, 2.0 * n_rot * d * 2, "GB/s", peaks["hbm"], f"{peaks['source']} hbm_gbs")
     rot["rows_per_call"] = n_rot
-    rec.update(queries=lblk, keys=T, note="includes the raw store of the block into its ring "
-               "slot (the append); sinks read from the rotated copy")
+    rec.update(queries=lblk, keys=T, scratch_bytes=n_scr,
+               note="includes the raw store of the block into its ring slot (the append); "
+                    "sinks read from the rotated copy")
     return rec, rot
 
 
@@ -387,6 +392,8 @@ def kernel_records(st, args):
         rec[f"attention_{name}"] = attention_alone(name, w, k)
         rec[f"attention_{name}_split"] = attention_alone(name, w, k, split=True)
     rec["attention_fused_480x480"], rec["rotate_ring_slots_480x480"] = fused_alone("480x480", w, k)
+    for name in ("384x672", "384x672_r4", "672x384"):
+        rec[f"attention_fused_{name}_split"] = fused_alone(name, w, k, split=True)[0]
     rec["note"] = ("attention: burst bf16 peak (a kernel timed alone); 'rotating' alternates "
                    "two input sets of 322 MB, 'repeat' reuses one (K/V of 295 MB exceed the "
                    "126 MB L2 either way)")
