@@ -225,17 +225,19 @@ def _summary(ms, work, unit, peak, peak_source):
 
 
 def attention_alone(name: str, warmup: int, steps: int, repeat: bool = False, nbuf: int = 2,
-                    split: bool = False):
+                    split: bool = False, heads: int = None):
     """One attention call at a workload's full size (block 1000, every slot valid), timed
     alone.  ``repeat`` = the same inputs every launch; otherwise ``nbuf`` input sets (each
     larger than L2) alternate.  ``split``: prsink_attention_split (the last wave's units split
-    over the key range)."""
+    over the key range).  ``heads``: fewer heads than the workload's (an L2-resident case)."""
     import torch
 
     import pose_retrieved_kv_b200 as P
     import synth
 
     cfg = synth.preset(name, block_index=1000, valid_mask=0xFF)
+    if heads is not None:
+        cfg["n_heads"] = heads
     lay = P.make_layout(**cfg)
     _, lblk, _, T = P.prsink_layout_tokens(lay)
     H, d = cfg["n_heads"], cfg["head_dim"]
@@ -391,12 +393,18 @@ def kernel_records(st, args):
     for name in ("384x672", "384x672_r4", "672x384"):
         rec[f"attention_{name}"] = attention_alone(name, w, k)
         rec[f"attention_{name}_split"] = attention_alone(name, w, k, split=True)
+    # hot against cold L2 at 13 heads (143 units: one wave of 148 SMs): 105 MB of Q/K/V stay
+    # resident when repeated; three alternating sets (315 MB) do not
+    rec["attention_480x480_13heads_hot_l2"] = attention_alone("480x480", w, k, repeat=True,
+                                                              heads=13)
+    rec["attention_480x480_13heads_cold_l2"] = attention_alone("480x480", w, k, nbuf=3, heads=13)
     rec["attention_fused_480x480"], rec["rotate_ring_slots_480x480"] = fused_alone("480x480", w, k)
     for name in ("384x672", "384x672_r4", "672x384"):
         rec[f"attention_fused_{name}_split"] = fused_alone(name, w, k, split=True)[0]
     rec["note"] = ("attention: burst bf16 peak (a kernel timed alone); 'rotating' alternates "
                    "two input sets of 322 MB, 'repeat' reuses one (K/V of 295 MB exceed the "
-                   "126 MB L2 either way)")
+                   "126 MB L2 either way); the 13-head pair compares L2-resident inputs (hot) "
+                   "with three alternating sets (cold)")
     return rec
 
 
